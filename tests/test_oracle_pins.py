@@ -1,0 +1,364 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Nothing here re-types the oracle's own formulas: every check compares it to
+a closed form, a hand-derived fixture (tests/golden), a library routine
+(scipy's Sylvester Hadamard matrix, numpy's little-endian bit packing,
+torch's scaled_dot_product_attention in fp64) or an invariant of the
+method (orthonormality, rotation invariance of exact attention, the
+quantiser's error bound, power-of-two and sign equivariance, causality).
+"""
+import math
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import oracle
+from conftest import read_golden
+from quantized_paged_kv_tq_b200 import workloads as W
+
+BITS = (2, 3, 4, 8)
+
+
+def Lof(b):
+    return (1 << (b - 1)) - 1
+
+
+def rand_bf16(rng, shape, scale=1.0):
+    return W.f32_to_bf16_bits(rng.standard_normal(shape).astype(np.float32) * scale)
+
+
+# --------------------------------------------------------------------- WHT
+@pytest.mark.parametrize("d", [2, 4, 8, 16, 32, 64, 128])
+def test_fwht_is_sylvester_hadamard(d):
+    """Columns of the oracle's transform are the Sylvester Hadamard matrix:
+    scipy.linalg.hadamard and the closed form (-1)^popcount(i & j)."""
+    H32 = np.stack([oracle.fwht_f32(np.eye(d, dtype=np.float32)[j]) for j in range(d)], 1)
+    H64 = np.stack([oracle.fwht_f64(np.eye(d)[j]) for j in range(d)], 1)
+    ref = scipy.linalg.hadamard(d)
+    i, j = np.meshgrid(np.arange(d), np.arange(d), indexing="ij")
+    closed = np.where(np.vectorize(lambda a: bin(a).count("1") % 2)(i & j), -1, 1)
+    assert np.array_equal(H32, ref) and np.array_equal(H64, ref)
+    assert np.array_equal(ref, closed)
+    # H H = d I exactly
+    assert np.array_equal(H64 @ H64, d * np.eye(d))
+
+
+def test_fwht_golden_h4():
+    rows = np.array(read_golden("hadamard_d4.txt"), dtype=np.int64)
+    H = np.stack([oracle.fwht_f64(np.eye(4)[j]) for j in range(4)], 1)
+    assert np.array_equal(H, rows)
+
+
+def test_rotate_d2_closed_form():
+    """d = 2: y = [[1, 1], [1, -1]] x / sqrt(2)."""
+    for a, b in [(1.0, 0.5), (-3.0, 2.0), (0.25, 0.25)]:
+        x = W.f32_to_bf16_bits(np.array([a, b], np.float32))
+        y = oracle.rotate_f32(x)
+        assert np.allclose(y, [(a + b) / math.sqrt(2), (a - b) / math.sqrt(2)],
+                           rtol=2e-7, atol=0)
+
+
+def test_rotation_matches_fp64_hadamard_and_preserves_norm():
+    rng = np.random.default_rng(5)
+    H = scipy.linalg.hadamard(128).astype(np.float64)
+    for _ in range(50):
+        x = rand_bf16(rng, 128, scale=rng.uniform(0.01, 30))
+        xf = W.bf16_bits_to_f32(x).astype(np.float64)
+        y = oracle.rotate_f32(x).astype(np.float64)
+        ref = H @ xf / math.sqrt(128)
+        assert np.max(np.abs(y - ref)) <= 8 * 2.0 ** -24 * np.max(np.abs(ref)) * 8
+        assert abs(np.linalg.norm(y) / np.linalg.norm(xf) - 1.0) < 1e-6
+
+
+# --------------------------------------------------------------- quantiser
+def test_golden_e0_codes():
+    """x = e_0: every rotated entry is fp32(1/sqrt(128)), so every code is +L."""
+    x = np.zeros(128, np.uint16)
+    x[0] = 0x3F80  # bf16 1.0
+    for bits_s, scale_hex, pattern in read_golden("quant_e0.txt"):
+        bits = int(bits_s)
+        packed, s = oracle.quantize_vector(x, bits)
+        assert np.float32(s).view(np.uint32) == int(scale_hex, 16)
+        pat = bytes.fromhex(pattern)
+        assert packed.tobytes() == pat * (len(packed) // len(pat))
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_constant_vector_exact(bits):
+    """x = a * 1: the rotation concentrates everything in y_0 = a sqrt(d)
+    (exactly, in fp32), so code_0 = sign(a) L and every other code is 0."""
+    for a in (1.0, -2.5, 0.375):
+        x = W.f32_to_bf16_bits(np.full(128, a, np.float32))
+        y = oracle.rotate_f32(x)
+        assert y[0] == np.float32(np.float32(128 * a) * np.float32(1 / math.sqrt(128)))
+        assert np.all(y[1:] == 0)
+        codes, s = oracle.quantize_rotated(y, bits)
+        assert codes[0] == (Lof(bits) if a > 0 else -Lof(bits))
+        assert np.all(codes[1:] == 0)
+        assert s == abs(y[0])
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_dequant_error_bound(bits):
+    """|code s / L - y| <= s / (2L) for every element (plus fp32 slack)."""
+    rng = np.random.default_rng(bits)
+    L = Lof(bits)
+    for _ in range(200):
+        x = rand_bf16(rng, 128, scale=rng.uniform(0.1, 10))
+        x_f = W.bf16_bits_to_f32(x)
+        x_f[rng.choice(128, 3, replace=False)] *= 20
+        x = W.f32_to_bf16_bits(x_f)
+        y = oracle.rotate_f32(x).astype(np.float64)
+        codes, s = oracle.quantize_rotated(y.astype(np.float32), bits)
+        assert s == np.max(np.abs(y))
+        assert np.all(np.abs(codes) <= L)
+        err = np.abs(codes * float(s) / L - y)
+        assert np.all(err <= float(s) / (2 * L) * (1 + 2.0 ** -20))
+        # the absmax element is represented exactly by +-L
+        i = int(np.argmax(np.abs(y)))
+        assert abs(codes[i]) == L
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_pow2_scale_equivariance(bits):
+    """x * 2^k gives identical codes and scale * 2^k (bit-exact)."""
+    rng = np.random.default_rng(10 + bits)
+    for _ in range(50):
+        x = rand_bf16(rng, 128)
+        p0, s0 = oracle.quantize_vector(x, bits)
+        for k in (-3, 1, 5):
+            xk = W.f32_to_bf16_bits(W.bf16_bits_to_f32(x) * np.float32(2.0 ** k))
+            pk, sk = oracle.quantize_vector(xk, bits)
+            assert np.array_equal(p0, pk)
+            assert sk == np.float32(s0 * np.float32(2.0 ** k))
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_sign_symmetry(bits):
+    rng = np.random.default_rng(20 + bits)
+    for _ in range(50):
+        x = rand_bf16(rng, 128)
+        neg = x ^ np.uint16(0x8000)
+        y, yn = oracle.rotate_f32(x), oracle.rotate_f32(neg)
+        c, s = oracle.quantize_rotated(y, bits)
+        cn, sn = oracle.quantize_rotated(yn, bits)
+        assert s == sn and np.array_equal(c, -cn)
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_zero_vector(bits):
+    packed, s = oracle.quantize_vector(np.zeros(128, np.uint16), bits)
+    assert s == 0.0
+    assert np.array_equal(oracle.unpack_codes(packed, 128, bits), np.zeros(128))
+
+
+def test_round_half_away_from_zero_at_ties():
+    """Constructed ties: with s a multiple of L chosen so that y*L/s is exact,
+    n + 1/2 rounds away from zero."""
+    y = np.zeros(128, np.float32)
+    y[:6] = [7.0, 2.5, -2.5, 0.5, -0.5, 1.5]
+    c, s = oracle.quantize_rotated(y, 4)                      # L = 7, s = 7
+    assert s == 7 and list(c[:6]) == [7, 3, -3, 1, -1, 2]
+    y = np.zeros(128, np.float32)
+    y[:4] = [1.0, 0.5, -0.5, 0.25]
+    c, s = oracle.quantize_rotated(y, 2)                      # L = 1
+    assert list(c[:4]) == [1, 1, -1, 0]
+    y = np.zeros(128, np.float32)
+    y[:4] = [3.0, 0.5, -1.5, 2.5]
+    c, s = oracle.quantize_rotated(y, 3)                      # L = 3
+    assert list(c[:4]) == [3, 1, -2, 3]
+    y = np.zeros(128, np.float32)
+    y[:3] = [127.0, 2.5, -126.5]
+    c, s = oracle.quantize_rotated(y, 8)                      # L = 127
+    assert list(c[:3]) == [127, 3, -127]
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_packing_matches_numpy_little_endian_bits(bits):
+    rng = np.random.default_rng(30 + bits)
+    L = Lof(bits)
+    for _ in range(50):
+        codes = rng.integers(-L, L, size=128, endpoint=True).astype(np.int32)
+        u = (codes + L).astype(np.uint32)
+        bitmat = ((u[:, None] >> np.arange(bits)) & 1).astype(np.uint8)
+        ref = np.packbits(bitmat.ravel(), bitorder="little")
+        got = oracle.pack_codes(codes, bits)
+        assert np.array_equal(got, ref)
+        assert np.array_equal(oracle.unpack_codes(got, 128, bits), codes)
+
+
+def test_packing_golden():
+    for bits_s, codes_s, hexbytes in read_golden("pack_examples.txt"):
+        bits = int(bits_s)
+        codes = np.array([int(c) for c in codes_s.split(",")], np.int32)
+        assert oracle.pack_codes(codes, bits).tobytes() == bytes.fromhex(hexbytes)
+
+
+def test_compression_ratio_turbo4():
+    """The page's compression table gives 3.7x for turbo4 over BF16 ("TurboQuant
+    is a memory trade"; xinfer-ai performance tips: "turbo4 gives 3.7x
+    compression"): 256 B of bf16 vs 64 B of 4-bit codes + a 4 B fp32 scale."""
+    bf16 = oracle.block_bytes(16, 128, 16)
+    t4 = oracle.block_bytes(4, 128, 16)
+    assert bf16 == 16 * 256 and t4 == 16 * 68
+    assert abs(bf16 / t4 - 3.7) < 0.1
+
+
+# --------------------------------------------------------------- attention
+def _sdpa(q, K, V, causal_last):
+    """torch fp64 SDPA of rows q [R][d] over K/V [n][d]; row r sees keys
+    0..causal_last[r]."""
+    n = K.shape[0]
+    mask = torch.tensor(np.arange(n)[None, :] <= np.asarray(causal_last)[:, None])
+    return torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q)[None], torch.tensor(K)[None], torch.tensor(V)[None],
+        attn_mask=mask[None]).numpy()[0]
+
+
+def _pools(w, fmt):
+    bb = oracle.block_bytes(fmt, w.head_dim, w.page_size)
+    if fmt == 16:
+        shape = (w.num_pages, w.num_kv_heads, w.page_size, w.head_dim)
+        return np.zeros(shape, np.uint16), np.zeros(shape, np.uint16)
+    shape = (w.num_pages, w.num_kv_heads, bb)
+    return np.zeros(shape, np.uint8), np.zeros(shape, np.uint8)
+
+
+def _fill(w, fmt):
+    kp, vp = _pools(w, fmt)
+    for slots, k, v in w.iter_fill():
+        if fmt == 16:
+            oracle.append_bf16(k, v, slots, w.page_size, kp, vp)
+        else:
+            oracle.quantize_append(k, v, slots, fmt, w.page_size, kp, vp)
+    return kp, vp
+
+
+def _dequant_numpy(pool, fmt, page, kvh, off, P, d=128):
+    """Rotated dequantised row via numpy's little-endian unpackbits."""
+    cb = d * fmt // 8
+    blk = pool[page, kvh]
+    bits = np.unpackbits(blk[off * cb:(off + 1) * cb], bitorder="little")
+    u = (bits.reshape(d, fmt) * (1 << np.arange(fmt))).sum(1)
+    s = blk[P * cb + 4 * off:P * cb + 4 * off + 4].view(np.float32)[0]
+    L = Lof(fmt)
+    return (u - L) * float(s) / L
+
+
+@pytest.mark.parametrize("fmt", [16, 4, 3, 8, 2])
+@pytest.mark.parametrize("q_len", [1, 3])
+def test_paged_decode_matches_sdpa(fmt, q_len):
+    """The paged decode equals textbook softmax attention (torch SDPA, fp64)
+    on the de-rotated dequantised K/V gathered through the page table, with
+    the causal limit j <= seq_len - q_len + t and GQA group h // group."""
+    w = W.custom(batch=3, num_q_heads=6, num_kv_heads=2, page_size=16,
+                 q_len=q_len, seq_lens=(37, 16, 5 + q_len), fmt=fmt, seed=fmt)
+    kp, vp = _fill(w, fmt)
+    q = w.queries()
+    out = oracle.paged_decode(q, fmt, w.page_size, kp, vp, w.page_table,
+                              w.seq_lens, w.num_kv_heads)
+    H = scipy.linalg.hadamard(128) / math.sqrt(128)
+    P = w.page_size
+    for b in range(w.batch):
+        n = int(w.seq_lens[b])
+        for h in range(w.num_q_heads):
+            kvh = h // w.group
+            K = np.zeros((n, 128))
+            V = np.zeros((n, 128))
+            for j in range(n):
+                page, off = int(w.page_table[b, j // P]), j % P
+                if fmt == 16:
+                    K[j] = W.bf16_bits_to_f32(kp[page, kvh, off])
+                    V[j] = W.bf16_bits_to_f32(vp[page, kvh, off])
+                else:
+                    K[j] = H @ _dequant_numpy(kp, fmt, page, kvh, off, P)
+                    V[j] = H @ _dequant_numpy(vp, fmt, page, kvh, off, P)
+            qr = W.bf16_bits_to_f32(q[b, :, h]).astype(np.float64)
+            ref = _sdpa(qr, K, V, [n - q_len + t for t in range(q_len)])
+            assert np.max(np.abs(out[b, :, h] - ref)) < 1e-11
+
+
+def test_rotation_invariance_of_exact_attention():
+    """Attending in the Hadamard basis (q, K, V rotated, output rotated back)
+    equals plain attention when nothing is quantised."""
+    rng = np.random.default_rng(40)
+    for n in (1, 7, 300):
+        q = rng.standard_normal(128)
+        K = rng.standard_normal((n, 128)) * 2
+        V = rng.standard_normal((n, 128))
+        Kr = np.stack([oracle.fwht_f64(k) / math.sqrt(128) for k in K])
+        Vr = np.stack([oracle.fwht_f64(v) / math.sqrt(128) for v in V])
+        a = oracle.attention_f64(q, K, V, rotated=False)
+        b = oracle.attention_f64(q, Kr, Vr, rotated=True)
+        assert np.max(np.abs(a - b)) < 1e-5
+        assert np.max(np.abs(a - b)) < 1e-12
+
+
+def test_single_key_and_identical_keys():
+    rng = np.random.default_rng(41)
+    q = rng.standard_normal(128)
+    v = rng.standard_normal(128)
+    k = rng.standard_normal(128)
+    # one key: output is that value, whatever the score
+    assert np.allclose(oracle.attention_f64(q, k[None], v[None], False), v, atol=1e-15)
+    vr = oracle.fwht_f64(v) / math.sqrt(128)
+    assert np.allclose(oracle.attention_f64(q, k[None], vr[None], True), v, atol=1e-13)
+    # identical keys: output is the mean of the values
+    V = rng.standard_normal((9, 128))
+    K = np.repeat(k[None], 9, 0)
+    assert np.allclose(oracle.attention_f64(q, K, V, False), V.mean(0), atol=1e-14)
+
+
+def test_brute_force_softmax_tiny():
+    """Explicit exp/sum on a 4-dimensional, 3-key case."""
+    q = np.array([0.5, -1.0, 2.0, 0.0])
+    K = np.array([[1.0, 0, 0, 0], [0, 1.0, 0, 0], [0, 0, 1.0, 1.0]])
+    V = np.array([[1.0, 2, 3, 4], [-1.0, 0, 1, 0], [0.0, 0, 0, 8]])
+    s = [0.5 / 2, -1.0 / 2, 2.0 / 2]
+    e = [math.exp(x) for x in s]
+    ref = sum(ei * V[i] for i, ei in enumerate(e)) / sum(e)
+    assert np.allclose(oracle.attention_f64(q, K, V, False), ref, atol=1e-15)
+
+
+@pytest.mark.parametrize("fmt", [4, 16])
+def test_causal_rows_equal_shorter_single_token_decode(fmt):
+    """Row t of a q_len = 4 verify equals a q_len = 1 decode of the same
+    query at seq_len - 3 + t."""
+    w = W.custom(batch=2, num_q_heads=4, num_kv_heads=1, q_len=4,
+                 seq_lens=(50, 21), fmt=fmt, seed=7)
+    kp, vp = _fill(w, fmt)
+    q = w.queries()
+    out = oracle.paged_decode(q, fmt, w.page_size, kp, vp, w.page_table,
+                              w.seq_lens, w.num_kv_heads)
+    for t in range(4):
+        lens = w.seq_lens - 3 + t
+        single = oracle.paged_decode(np.ascontiguousarray(q[:, t:t + 1]), fmt,
+                                     w.page_size, kp, vp, w.page_table, lens,
+                                     w.num_kv_heads)
+        assert np.array_equal(single[:, 0], out[:, t])
+
+
+def test_quantize_append_layout_and_skip():
+    """Appended rows land at block (page, head), row `offset`, scale after
+    the codes; slot -1 writes nothing."""
+    rng = np.random.default_rng(50)
+    k = rand_bf16(rng, (3, 2, 128))
+    v = rand_bf16(rng, (3, 2, 128))
+    kp = np.zeros((4, 2, oracle.block_bytes(4, 128, 16)), np.uint8)
+    vp = np.zeros_like(kp)
+    oracle.quantize_append(k, v, np.array([5, -1, 16 * 3 + 15]), 4, 16, kp, vp)
+    for t, (page, off) in ((0, (0, 5)), (2, (3, 15))):
+        for h in range(2):
+            pk, sk = oracle.quantize_vector(k[t, h], 4)
+            pv, sv = oracle.quantize_vector(v[t, h], 4)
+            assert np.array_equal(kp[page, h, off * 64:(off + 1) * 64], pk)
+            assert np.array_equal(vp[page, h, off * 64:(off + 1) * 64], pv)
+            assert kp[page, h, 1024 + 4 * off:1028 + 4 * off].view(np.float32)[0] == sk
+            assert vp[page, h, 1024 + 4 * off:1028 + 4 * off].view(np.float32)[0] == sv
+    written = {(0, 5), (3, 15)}
+    for page in range(4):
+        for off in range(16):
+            if (page, off) not in written:
+                assert not kp[page, :, off * 64:(off + 1) * 64].any()
