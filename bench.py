@@ -1,0 +1,460 @@
+"""Benchmark of the TurboQuant paged KV path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload target64x8k] [--fmt 4]
+
+One step = append one new token per sequence (tq_quantize_append) + one
+decode over the whole paged cache (tq_paged_decode), on the workload named in
+``config.workload``.  Inputs are resident in HBM when the timed region
+starts; the cache (570 MB for the default workload) is larger than L2, so no
+flush is needed between steps.  ``value`` is the effective KV bandwidth of
+the step (algorithmic cache bytes read per step / step time); the line also
+carries seq/s, the append bandwidth, a roofline object for the decode
+kernel, an end-to-end number through the C ABI with host buffers, the
+oracle as a CPU baseline, and the SM clocks seen during the timed region.
+
+With --gpus N (launched by torch.distributed.run) every rank runs an
+independent replica on its own GPU: the workload has no exchange step, so
+there is no collective on the data path; only the timings are reduced (max
+over ranks).  ``--impl reference`` times the CPU oracle instead (rank 0
+only).
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from quantized_paged_kv_tq_b200 import workloads as W  # noqa: E402
+
+METRIC = "paged TurboQuant decode: effective KV GB/s (% of HBM peak), seq/s; append GB/s"
+DEFAULT_WORKLOAD = "target64x8k"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def describe(w: W.Workload, fmt: int) -> str:
+    names = {2: "turbo2", 3: "turbo3", 4: "turbo4", 8: "turbo8", 16: "bf16"}
+    lens = (f"{int(w.seq_lens[0])} tokens" if np.all(w.seq_lens == w.seq_lens[0])
+            else f"lengths {int(w.seq_lens.min())}-{int(w.seq_lens.max())}")
+    return (f"{w.name}: batch {w.batch} x {lens}, {w.num_q_heads} q / {w.num_kv_heads} kv "
+            f"heads, head_dim {w.head_dim}, page {w.page_size}, {names[fmt]}, q_len {w.q_len}; "
+            f"each step appends 1 token per sequence then decodes")
+
+
+def step_bytes(w: W.Workload, fmt: int):
+    kv = w.tokens_read() * 2 * W.row_bytes(fmt)                 # K and V rows read
+    new = w.batch * w.num_kv_heads * 2
+    append = new * (2 * w.head_dim + W.row_bytes(fmt)) + w.batch * 8
+    return kv, append
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+
+
+def profiled_traffic(kernel: str):
+    """dram read+write bytes per launch recorded in profiles/<kernel>*.txt,
+    valid only while decode.cu is unchanged (its sha256 is recorded too)."""
+    src = os.path.join(ROOT, "quantized_paged_kv_tq_b200", "csrc", "decode.cu")
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    pdir = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(pdir):
+        return None
+    for name in sorted(os.listdir(pdir)):
+        if not name.startswith(kernel):
+            continue
+        vals = {}
+        with open(os.path.join(pdir, name)) as f:
+            for line in f:
+                if ":" in line:
+                    k, v = line.split(":", 1)
+                    vals[k.strip()] = v.strip()
+        if vals.get("decode_cu_sha256") == sha and "traffic_bytes_per_launch" in vals:
+            return float(vals["traffic_bytes_per_launch"])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu: int):
+        self.gpu = gpu
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for r in csv.reader(f):
+                if len(r) >= 9:
+                    rows.append([x.strip() for x in r])
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------ CPU oracle
+def oracle_sample_decode(w: W.Workload, fmt: int, ntok: int, kv_head: int = 0, seq: int = 0):
+    """Time the CPU oracle decoding one (sequence, kv head): the first `ntok`
+    tokens of sequence `seq`, its `group` query heads, from a cache the
+    oracle builds itself (untimed).  Returns (seconds, algorithmic bytes)."""
+    import oracle
+    P = w.page_size
+    npages = (ntok + P - 1) // P
+    phys = w.page_table[seq, :npages].astype(np.int64)
+    slots = (phys[:, None] * P + np.arange(P)[None, :]).ravel()
+    k, v = w.kv_for_slots(slots)
+    k = np.ascontiguousarray(k[:, kv_head:kv_head + 1])
+    v = np.ascontiguousarray(v[:, kv_head:kv_head + 1])
+    bb = oracle.block_bytes(fmt, w.head_dim, P)
+    if fmt == 16:
+        kp = np.zeros((npages, 1, P, w.head_dim), np.uint16)
+        vp = np.zeros_like(kp)
+        oracle.append_bf16(k, v, np.arange(npages * P), P, kp, vp)
+    else:
+        kp = np.zeros((npages, 1, bb), np.uint8)
+        vp = np.zeros_like(kp)
+        oracle.quantize_append(k, v, np.arange(npages * P), fmt, P, kp, vp)
+    q = w.queries()[seq:seq + 1, :, kv_head * w.group:(kv_head + 1) * w.group]
+    pt = np.arange(npages, dtype=np.int32)[None]
+    t0 = time.perf_counter()
+    oracle.paged_decode(np.ascontiguousarray(q), fmt, P, kp, vp, pt,
+                        np.array([ntok], np.int32), 1)
+    dt = time.perf_counter() - t0
+    return dt, ntok * 2 * W.row_bytes(fmt)
+
+
+def cpu_baseline(w, fmt, budget_s=12.0):
+    """The oracle, single-threaded, on a bounded sample of the workload."""
+    n, secs, nbytes = 0, 0.0, 0
+    ntok = int(w.seq_lens[0])
+    while secs < budget_s and n < w.batch * w.num_kv_heads:
+        seq, kvh = divmod(n, w.num_kv_heads)
+        dt, b = oracle_sample_decode(w, fmt, min(ntok, int(w.seq_lens[seq])), kvh, seq)
+        secs += dt
+        nbytes += b
+        n += 1
+    return {"value": nbytes / secs / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} (sequence, kv head) decodes of up to {ntok} tokens x {w.group} "
+                      f"q heads each ({nbytes / 1e6:.1f} MB of cache), single-threaded C, "
+                      f"{os.cpu_count()} host cores present",
+            "seconds": secs}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = W.make(args.workload)
+    fmt = args.fmt or w.formats[0]
+    budget = 90.0
+    # calibrate the per-step sample so the whole run stays within ~budget
+    dt, b = oracle_sample_decode(w, fmt, 1024)
+    per_tok = dt / 1024
+    ntok = int(max(16, min(int(w.seq_lens[0]), budget / (args.steps + args.warmup) / per_tok)))
+    ntok = (ntok // 16) * 16
+    for i in range(args.warmup):
+        oracle_sample_decode(w, fmt, ntok, i % w.num_kv_heads)
+    secs, nbytes = 0.0, 0
+    for i in range(args.steps):
+        dt, b = oracle_sample_decode(w, fmt, ntok, i % w.num_kv_heads)
+        secs += dt
+        nbytes += b
+    value = nbytes / secs / 1e9
+    line = {"metric": METRIC, "impl": "reference", "value": value, "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": describe(w, fmt), "global_batch": w.batch,
+                       "seq_len": int(w.seq_lens.max()), "parallelism": "cpu-1thread"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"each step: one (sequence, kv head) decode over "
+                                       f"{ntok} tokens x {w.group} q heads, single-threaded C"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------- GPU arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (libtq.so has no CPU path)")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    from quantized_paged_kv_tq_b200 import build as tqbuild
+    tqbuild.build()
+    from quantized_paged_kv_tq_b200 import tq
+
+    w = W.make(args.workload)
+    fmt = args.fmt or w.formats[0]
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    def d_bf16(u16):
+        return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+
+    # ---- resident cache: every context token but the last of each sequence
+    cache = tq.Cache(fmt, w.num_pages, w.num_kv_heads, w.page_size, device=dev)
+    ctx = w.seq_lens - 1
+    for slots, k, v in w.iter_fill(upto=ctx):
+        ks, vs = d_bf16(k), d_bf16(v)
+        ss = torch.from_numpy(slots.astype(np.int64)).to(dev)
+        if fmt == 16:
+            tq.tq_append_bf16(ks, vs, ss, cache)
+        else:
+            tq.tq_quantize_append(ks, vs, ss, fmt, cache)
+    # per-step inputs: a few distinct new-token sets, appended at position
+    # seq_len - 1 of every sequence
+    n_variants = 4
+    new_slots = torch.from_numpy(np.array([w.slots_of(b, [int(w.seq_lens[b]) - 1])[0]
+                                           for b in range(w.batch)], np.int64)).to(dev)
+    new_k, new_v = [], []
+    for i in range(n_variants):
+        k, v = w.new_tokens(i, w.batch)
+        new_k.append(d_bf16(k))
+        new_v.append(d_bf16(v))
+    q = d_bf16(w.queries())
+    pt = torch.from_numpy(w.page_table).to(dev)
+    sl = torch.from_numpy(w.seq_lens).to(dev)
+    out = torch.empty((w.batch, w.q_len, w.num_q_heads, w.head_dim), dtype=torch.float32,
+                      device=dev)
+    max_len = w.max_seq_len
+    ws = cache.workspace(w.batch, w.q_len, w.num_q_heads, max_len)
+    decode = tq.tq_paged_decode_bf16 if fmt == 16 else tq.tq_paged_decode
+
+    def append(i):
+        j = i % n_variants
+        if fmt == 16:
+            tq.tq_append_bf16(new_k[j], new_v[j], new_slots, cache)
+        else:
+            tq.tq_quantize_append(new_k[j], new_v[j], new_slots, fmt, cache)
+
+    def dec():
+        decode(q, cache, pt, sl, w.q_len, out, max_seq_len=max_len, workspace=ws)
+
+    torch.cuda.synchronize()
+
+    # ---- in-run HBM roofline probes (untimed region)
+    nbytes = 1 << 30
+    a = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    bbuf = torch.empty_like(a)
+    sink = torch.zeros(1, dtype=torch.int32, device=dev)
+    copy_ms, read_ms = [], []
+    for _ in range(3):
+        tq.tq_hbm_copy(a, bbuf)
+        tq.tq_hbm_read(a, sink)
+    for _ in range(10):
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record()
+        tq.tq_hbm_copy(a, bbuf)
+        e1.record()
+        tq.tq_hbm_read(a, sink)
+        e2.record()
+        e2.synchronize()
+        copy_ms.append(e0.elapsed_time(e1))
+        read_ms.append(e1.elapsed_time(e2))
+    copy_gbs = 2 * nbytes / (min(copy_ms) * 1e-3) / 1e9
+    read_gbs = nbytes / (min(read_ms) * 1e-3) / 1e9
+    del a, bbuf
+    torch.cuda.synchronize()
+
+    # ---- warm-up
+    for i in range(args.warmup):
+        append(i)
+        dec()
+    torch.cuda.synchronize()
+
+    # ---- timed region (device time, CUDA events on the launching stream)
+    K = args.steps
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_c = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(K):
+        ev_a[i].record(stream)
+        append(i)
+        ev_b[i].record(stream)
+        dec()
+        ev_c[i].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    total_ms = ev_a[0].elapsed_time(ev_c[-1])
+    append_ms = [ev_a[i].elapsed_time(ev_b[i]) for i in range(K)]
+    decode_ms = [ev_b[i].elapsed_time(ev_c[i]) for i in range(K)]
+
+    # ---- end to end through the C ABI with host buffers
+    e2e_steps = max(3, min(K, 200))
+    h_q = torch.empty(q.shape, dtype=q.dtype, pin_memory=True).copy_(q.cpu())
+    h_k = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True).copy_(x.cpu()) for x in new_k]
+    h_v = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True).copy_(x.cpu()) for x in new_v]
+    h_s = torch.empty(new_slots.shape, dtype=torch.int64, pin_memory=True).copy_(new_slots.cpu())
+    h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    d_q, d_k, d_v, d_s = (torch.empty_like(q), torch.empty_like(new_k[0]),
+                          torch.empty_like(new_v[0]), torch.empty_like(new_slots))
+    h2d = (h_q.numel() * 2 + h_k[0].numel() * 2 + h_v[0].numel() * 2 + h_s.numel() * 8)
+    d2h = h_out.numel() * 4
+
+    def e2e_step(i):
+        j = i % n_variants
+        d_q.copy_(h_q, non_blocking=True)
+        d_k.copy_(h_k[j], non_blocking=True)
+        d_v.copy_(h_v[j], non_blocking=True)
+        d_s.copy_(h_s, non_blocking=True)
+        if fmt == 16:
+            tq.tq_append_bf16(d_k, d_v, d_s, cache)
+        else:
+            tq.tq_quantize_append(d_k, d_v, d_s, fmt, cache)
+        decode(d_q, cache, pt, sl, w.q_len, out, max_seq_len=max_len, workspace=ws)
+        h_out.copy_(out, non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    err = cache.read_error()
+    if err:
+        raise SystemExit(f"device error word set: 0x{err:x}")
+
+    # ---- reduce over ranks: max of each time
+    ms_step = total_ms / K
+    dec_avg = sum(decode_ms) / K
+    app_avg = sum(append_ms) / K
+    if world > 1:
+        t = torch.tensor([ms_step, dec_avg, app_avg, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step, dec_avg, app_avg, e2e_ms = t.tolist()
+
+    kv_bytes, app_bytes = step_bytes(w, fmt)
+    peaks, peak_kind = measured_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    value = world * kv_bytes / (ms_step * 1e-3) / 1e9
+    achieved = kv_bytes / (dec_avg * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": describe(w, fmt), "global_batch": w.batch * world,
+                   "seq_len": int(w.seq_lens.max()), "parallelism": f"dp{world}",
+                   "l2": f"inputs larger than L2: {kv_bytes / 1e6:.0f} MB of cache read per "
+                         f"step vs 126 MB L2, no flush"},
+        "seq_per_s": world * w.batch / (ms_step * 1e-3),
+        "decode_kv_gbs": achieved,
+        "decode_ms": dec_avg,
+        "append_gbs": app_bytes / (app_avg * 1e-3) / 1e9,
+        "append_ms": app_avg,
+        "hbm_inrun_gbs": {"copy": copy_gbs, "read": read_gbs},
+        "frac_of_hbm": {"step": (value / world) / peak, "decode_kernel": achieved / peak,
+                        "decode_vs_inrun_copy": achieved / copy_gbs,
+                        "decode_vs_inrun_read": achieved / read_gbs},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": profiled_traffic("decode"),
+                     "peak_source": f"hbm_gbs of {peak_kind}",
+                     "algorithmic_bytes_per_launch": kv_bytes},
+        "e2e": {"value": world * kv_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * K,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, fmt)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=W.ALL)
+    ap.add_argument("--fmt", type=int, default=0, help="cache format (default: workload's first)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

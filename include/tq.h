@@ -1,0 +1,223 @@
+/*
+ * tq.h -- C ABI of libtq.so: TurboQuant paged KV cache on NVIDIA B200 (sm_100a).
+ *
+ * What it computes.  "xInfer: Pure-Rust LLM Inference Without a Python
+ * Runtime", section "What actually sits between the request and the tokens":
+ * the KV cache is compressed by a Walsh-Hadamard transform rotation followed
+ * by per-head absmax quantisation (a 2-4 bit cache; the --kvcache-dtype flag
+ * of section "Getting a server up" also offers turbo8, and no flag means BF16).
+ * Section "TurboQuant is a memory trade": reading the cache dequantises on
+ * every attention step.  "infero", section "Continuous batching": requests
+ * share the GPU over a paged KV cache.
+ *
+ * Arithmetic (the pages leave it open; this library fixes it):
+ *   rotation  y = H_d x / sqrt(d), H_d the Sylvester-ordered Hadamard matrix,
+ *             as fp32 butterflies with strides 1, 2, 4, ..., d/2 and then one
+ *             fp32 multiply by fp32(1/sqrt(d)); no fused multiply-add.
+ *   scale     s = max_i |y_i|, stored as fp32.
+ *   codes     L = 2^(b-1) - 1, code_i = clamp(roundf(fp32(y_i * L) / s), -L, L)
+ *             (IEEE division, ties away from zero); s == 0 gives all codes 0.
+ *   storage   u_i = code_i + L, bit-packed LSB-first: u_i occupies bits
+ *             [i*b, (i+1)*b) of a little-endian byte string of d*b/8 bytes.
+ *   attention dequantised yhat_i = code_i * s / L; score_j = (H q / sqrt(d)) .
+ *             yhat_k,j / sqrt(d); out = H (sum_j softmax_j yhat_v,j) / sqrt(d).
+ *             Query position t of q_len sees keys j <= seq_len - q_len + t.
+ *             Query head h reads kv head h / (num_q_heads / num_kv_heads).
+ *
+ * Cache layout in device memory (one pool for K, one for V, same shape):
+ *   pool[num_pages][num_kv_heads][block], block = tq_page_block_bytes(...).
+ *   turbo b-bit block: page_size rows of d*b/8 code bytes (row = token offset
+ *   within the page), then page_size fp32 scales.  BF16 block: page_size rows
+ *   of d bf16 values.  A token's slot is page * page_size + offset.
+ *
+ * Ownership.  The library allocates nothing and keeps no state between calls.
+ * Every buffer is caller-owned device memory unless stated otherwise.  Every
+ * call is asynchronous on the given CUDA stream (a cudaStream_t passed as
+ * void*, NULL = legacy default stream); calls on different streams are safe
+ * when their buffers are disjoint.
+ *
+ * Errors.  Arguments are checked on the host before anything is launched; a
+ * failed check returns a status and launches nothing.  A CUDA launch failure
+ * returns TQ_ERR_CUDA.  Problems only visible on the device (a page id or a
+ * slot outside the pool, a sequence length outside [q_len, max_seq_len], a
+ * bounded wait that expired) skip the affected work and record the first
+ * such event in the optional device word cache->dev_error; read it with
+ * tq_read_device_error.  No device code traps or asserts.
+ *
+ * Supported shapes: head_dim 128; page_size 16, 32 or 64; 1 <= q_len and
+ * q_len * (num_q_heads / num_kv_heads) <= 64.
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TQ_ABI_VERSION 1
+
+typedef enum {
+    TQ_OK = 0,
+    TQ_ERR_INVALID_ARG = 1,   /* bad pointer, size, shape or alignment */
+    TQ_ERR_UNSUPPORTED = 2,   /* well-formed but outside the supported shapes */
+    TQ_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+    TQ_ERR_TIMEOUT = 4,       /* a bounded device wait expired (device word) */
+    TQ_ERR_DEVICE_CHECK = 5,  /* a device-side range check failed (device word) */
+    TQ_ERR_WORKSPACE = 6      /* decode workspace missing or too small */
+} tq_status;
+
+/* KV cache formats: the --kvcache-dtype choices of the xInfer page (section
+ * "Getting a server up"; turbo2 extends its "2 to 4 bit" range downwards). */
+typedef enum {
+    TQ_TURBO2 = 2,
+    TQ_TURBO3 = 3,
+    TQ_TURBO4 = 4,
+    TQ_TURBO8 = 8,
+    TQ_BF16 = 16
+} tq_format;
+
+/* Descriptor of one layer's paged K/V pools.  Plain data; the pointed-to
+ * device memory is owned by the caller. */
+typedef struct {
+    int32_t format;        /* tq_format */
+    int32_t head_dim;      /* d; must be 128 */
+    int32_t num_kv_heads;  /* >= 1 */
+    int32_t page_size;     /* tokens per page: 16, 32 or 64 */
+    int32_t num_pages;     /* pages in each pool, >= 1 */
+    void* k_pages;         /* device, 16-byte aligned, num_pages*num_kv_heads*block bytes */
+    void* v_pages;         /* device, same size and alignment */
+    uint32_t* dev_error;   /* device word, optional (NULL: device findings dropped).
+                              0 = no error; else (tq_status) | (detail << 8). */
+} tq_cache;
+
+/* ABI version of the loaded library (TQ_ABI_VERSION). */
+int32_t tq_abi_version(void);
+
+/* Readable name of a status.  Never NULL; the string is static. */
+const char* tq_status_string(tq_status status);
+
+/* Bytes of one (page, kv head) block of a pool, per the layout above; 0 when
+ * the arguments are not a supported combination. */
+size_t tq_page_block_bytes(int32_t format, int32_t head_dim, int32_t page_size);
+
+/*
+ * tq_quantize_append -- rotate, absmax-quantise, bit-pack and store new K/V
+ * rows into a turbo cache ("What actually sits between the request and the
+ * tokens": Walsh-Hadamard rotation followed by per-head absmax quantisation).
+ *   k, v          device bf16 [num_tokens][num_kv_heads][head_dim], 16-byte
+ *                 aligned; one (token, head) row is one quantised vector.
+ *   slot_mapping  device int64 [num_tokens]: slot = page*page_size + offset;
+ *                 a negative slot skips the token; a slot past the pool is
+ *                 skipped and recorded as TQ_ERR_DEVICE_CHECK.
+ *   num_tokens    >= 0 (0 is a no-op).
+ *   bits          2, 3, 4 or 8; must equal cache->format.
+ * Result: codes and the fp32 scale of every (token, head) of K and of V are
+ * written at their slot; nothing else in the pools changes.  Bit-exact with
+ * the definition above for every finite input.
+ */
+tq_status tq_quantize_append(const void* k, const void* v,
+                             const int64_t* slot_mapping, int32_t num_tokens,
+                             int32_t bits, const tq_cache* cache, void* stream);
+
+/*
+ * tq_append_bf16 -- store new K/V rows unchanged into a BF16 cache (the
+ * "no flag means BF16" cache of "Getting a server up"), the uncompressed
+ * reference point.  Arguments as tq_quantize_append; cache->format must be
+ * TQ_BF16.
+ */
+tq_status tq_append_bf16(const void* k, const void* v,
+                         const int64_t* slot_mapping, int32_t num_tokens,
+                         const tq_cache* cache, void* stream);
+
+/*
+ * tq_decode_workspace_size -- bytes of device workspace tq_paged_decode and
+ * tq_paged_decode_bf16 need for these shapes (0 when every sequence fits in
+ * one split and none is needed).  The workspace holds per-split softmax
+ * partials and one merge counter per (sequence, kv head, row group).
+ * Returns 0 for invalid arguments as well; the decode call re-checks.
+ */
+size_t tq_decode_workspace_size(int32_t batch, int32_t q_len,
+                                int32_t num_q_heads, int32_t max_seq_len,
+                                const tq_cache* cache);
+
+/*
+ * tq_decode_workspace_init -- zero the merge counters of a workspace.  Call
+ * once after allocating it; every decode call leaves them zero again.
+ */
+tq_status tq_decode_workspace_init(void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
+/*
+ * tq_paged_decode -- batched decode / short speculative-verify attention over
+ * a turbo cache through per-sequence page tables, dequantising on the fly
+ * ("TurboQuant is a memory trade": dequantisation on every attention step;
+ * infero "Continuous batching": paged KV shared by a running batch).
+ *   q                device bf16 [batch][q_len][num_q_heads][head_dim].
+ *   page_table       device int32 [batch][max_pages_per_seq]; entry p is the
+ *                    physical page of tokens [p*page_size, (p+1)*page_size).
+ *                    Pages may be shared between sequences (prefix sharing).
+ *   seq_lens         device int32 [batch]: cached tokens of each sequence,
+ *                    the q_len new ones included (they must already be
+ *                    appended); q_len <= seq_lens[b] <= max_seq_len.
+ *   batch            >= 0 (0 is a no-op), <= 65535.
+ *   q_len            1 for decode, >1 for causal verify of draft tokens.
+ *   max_seq_len      host bound on seq_lens, sizes the launch and workspace.
+ *   out              device fp32 [batch][q_len][num_q_heads][head_dim],
+ *                    16-byte aligned; fully written for valid sequences.
+ *   workspace        device, tq_decode_workspace_size bytes (may be NULL
+ *                    when that size is 0), 16-byte aligned, initialised once
+ *                    by tq_decode_workspace_init.  Calls that overlap in
+ *                    time must use different workspaces.
+ * Each sequence is split into fixed 512-token (page_size 16/32) or
+ * 1024-token (page_size 64) parts whatever the batch holds, so a
+ * sequence's output does not depend on the other sequences of the batch.
+ */
+tq_status tq_paged_decode(const void* q, const tq_cache* cache,
+                          const int32_t* page_table, int32_t max_pages_per_seq,
+                          const int32_t* seq_lens, int32_t batch, int32_t q_len,
+                          int32_t num_q_heads, int32_t max_seq_len, float* out,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * tq_paged_decode_bf16 -- the same decode over a BF16 cache (no rotation, no
+ * scales): out = softmax(q k / sqrt(d)) v.  Arguments and workspace rules
+ * as tq_paged_decode; cache->format must be TQ_BF16.
+ */
+tq_status tq_paged_decode_bf16(const void* q, const tq_cache* cache,
+                               const int32_t* page_table,
+                               int32_t max_pages_per_seq,
+                               const int32_t* seq_lens, int32_t batch,
+                               int32_t q_len, int32_t num_q_heads,
+                               int32_t max_seq_len, float* out,
+                               void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/*
+ * tq_read_device_error -- wait (bounded, ~10 s) for the stream, then copy the
+ * device error word of cache->dev_error into *code (0 when no word is set);
+ * clear != 0 resets it to zero.  Returns TQ_ERR_TIMEOUT if the stream did
+ * not finish in time, TQ_ERR_CUDA on a CUDA failure, else TQ_OK.
+ */
+tq_status tq_read_device_error(const tq_cache* cache, uint32_t* code,
+                               int32_t clear, void* stream);
+
+/*
+ * Roofline probes used by the benchmark to measure this GPU's HBM bandwidth
+ * in the same run (no counterpart on the pages):
+ *   tq_hbm_copy  dst[i] = src[i] over `bytes` bytes (16-byte aligned,
+ *                bytes a multiple of 16); moves 2*bytes through HBM.
+ *   tq_hbm_read  reads `bytes` bytes and writes one 32-bit checksum to
+ *                *sink so the read cannot be elided; moves `bytes`.
+ */
+tq_status tq_hbm_copy(const void* src, void* dst, size_t bytes, void* stream);
+tq_status tq_hbm_read(const void* src, size_t bytes, uint32_t* sink,
+                      void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

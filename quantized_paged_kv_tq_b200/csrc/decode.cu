@@ -1,0 +1,912 @@
+// Paged decode / speculative-verify attention over a TurboQuant or bf16 cache.
+//
+// "xInfer: Pure-Rust LLM Inference Without a Python Runtime", section
+// "TurboQuant is a memory trade": reading a low-bit KV cache dequantises on
+// every attention step.  "infero", section "Continuous batching": a running
+// batch shares the GPU over a paged KV cache.
+//
+// Work decomposition (split-KV):
+//   grid = (max splits, kv heads x row groups, batch), 4 warps per CTA.
+//   A CTA owns one (sequence, kv head, row group, split); a split is a fixed
+//   run of 512 tokens (1024 for 64-token pages), so a sequence's result
+//   never depends on the rest of the batch.  All G = q_len * GQA query rows
+//   of the kv head (up to 8 per row group) share every byte read.
+//   Each warp streams its own 16-token tiles (tile w, w+4, ...) through a
+//   private ring of shared-memory stages filled by 1-D bulk async copies
+//   (cp.async.bulk + mbarrier; codes and fp32 scales of K and V).
+//
+// Per tile (16 tokens):
+//   QK^T  mma.sync m16n8k16, A = K codes unpacked in registers to exact f16
+//         integers (magic-number trick), B = the rotated query split into f16
+//         hi + lo parts (8 columns = 4 rows x {hi, lo}); fp32 accumulate.
+//         score = raw * (s_k / L) in log2 units.
+//   softmax online, with a lazy rescale: the running max only moves when a
+//         tile exceeds it by 2^8; causal limit j <= seq_len - q_len + t.
+//   PV    mma.sync with A = V codes (dims on M, tokens on K) and B = P' =
+//         p * s_v / L (hi + lo f16) transposed in registers by movmatrix.
+//         A running power-of-two V-scale exponent keeps P' inside f16 range.
+// Epilogue: the 4 warps merge in shared memory; a sequence with one split
+// finishes directly, otherwise the CTA stores (m, l, O) partials and the last
+// CTA of the (sequence, kv head, row group), found with an atomic ticket,
+// merges all splits, rotates back (H o / sqrt(d)) and writes fp32 output.
+#include <cstdint>
+#include <math_constants.h>
+
+#include "tq_device.cuh"
+
+namespace tq {
+
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kMaxStages = 4;
+constexpr int kRowsPerCta = 8;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLazyThreshold = 8.f;       // log2 units
+constexpr uint32_t kWaitSpins = 1u << 24;   // bounded mbarrier polls
+constexpr uint32_t kMagic = 0x64006400u;    // f16 pair (1024, 1024)
+
+struct DecodeArgs {
+    const uint16_t* q;
+    const uint8_t* kp;
+    const uint8_t* vp;
+    const int32_t* page_table;
+    const int32_t* seq_lens;
+    float* out;
+    float* ws_o;
+    float2* ws_ml;
+    uint32_t* ws_cnt;
+    uint32_t* err;
+    int64_t block_bytes;
+    int max_pages;
+    int num_pages;
+    int num_kv_heads;
+    int num_q_heads;
+    int group;
+    int q_len;
+    int G;          // query rows per kv head
+    int R;          // row groups of <= 8 rows
+    int page_size;
+    int split_tokens;
+    int max_splits;
+    int max_seq_len;
+    int stages;
+};
+
+template <int BITS>
+struct Fmt {
+    static constexpr bool kTurbo = BITS != 16;
+    static constexpr int CB = kTurbo ? kHeadDim * BITS / 8 : 2 * kHeadDim;  // row bytes
+    static constexpr int kTileCodes = 16 * CB;
+    static constexpr int kVOff = kTurbo ? kTileCodes + 64 : kTileCodes;
+    static constexpr int kStageBytes = 2 * kVOff;
+    static constexpr int L = kTurbo ? (1 << (BITS - 1)) - 1 : 1;
+};
+
+// QK^T tile row r (0..15) holds tile token perm(r); chosen so that the
+// transposed probabilities land on the PV B-fragment (tokens t, t+4, t+8,
+// t+12 for lane group t) and shared-memory reads spread over banks.
+__device__ __forceinline__ int perm(int r)
+{
+    return (r & 8) | ((r & 1) << 2) | ((r >> 1) & 3);
+}
+
+// Head dimension held by fragment element (chunk c, k = 2t + e + 8f) of the
+// QK^T operands; it follows the order the unpacker produces values in.
+template <int BITS>
+__device__ __forceinline__ int qk_dim(int t, int c, int f, int e)
+{
+    if constexpr (BITS == 4 || BITS == 3) return 32 * t + 8 * (c >> 1) + 2 * (c & 1) + f + 4 * e;
+    if constexpr (BITS == 8) return 32 * t + 4 * c + f + 2 * e;
+    if constexpr (BITS == 2) return 32 * t + 16 * (c >> 2) + 2 * (c & 3) + f + 8 * e;
+    return 32 * t + 8 * (c >> 1) + 4 * (c & 1) + 2 * f + e;  // bf16
+}
+
+// ----------------------------------------------------------- K unpackers
+// ka[c][f]: f16x2 (bf16x2) A-fragment element pair for chunk c, half f, of
+// one token row; `row` points at that token's code bytes in the stage.
+template <int BITS>
+__device__ __forceinline__ void unpack_k(const uint8_t* row, int t, uint32_t ka[8][2])
+{
+    if constexpr (BITS == 4) {
+        const uint4 w = *reinterpret_cast<const uint4*>(row + 16 * t);
+        const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi)
+#pragma unroll
+            for (int hb = 0; hb < 2; ++hb) {
+                const uint32_t x = hb ? words[wi] >> 8 : words[wi];
+                ka[2 * wi + hb][0] = hfma2_u32(and_or(x, 0x000F000Fu, kMagic), 0x3C003C00u, 0xE407E407u);
+                ka[2 * wi + hb][1] = hfma2_u32(and_or(x, 0x00F000F0u, kMagic), 0x2C002C00u, 0xD470D470u);
+            }
+    } else if constexpr (BITS == 8) {
+        const uint4 w0 = *reinterpret_cast<const uint4*>(row + 32 * t);
+        const uint4 w1 = *reinterpret_cast<const uint4*>(row + 32 * t + 16);
+        const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            ka[c][0] = hfma2_u32(prmt(words[c], 0x64646464u, 0x4240u), 0x3C003C00u, 0xE47FE47Fu);
+            ka[c][1] = hfma2_u32(prmt(words[c], 0x64646464u, 0x4341u), 0x3C003C00u, 0xE47FE47Fu);
+        }
+    } else if constexpr (BITS == 2) {
+        const uint2 w = *reinterpret_cast<const uint2*>(row + 8 * t);
+        const uint32_t words[2] = {w.x, w.y};
+        constexpr uint32_t mul[4] = {0x3C003C00u, 0x34003400u, 0x2C002C00u, 0x24002400u};
+        constexpr uint32_t add[4] = {0xE401E401u, 0xDC04DC04u, 0xD410D410u, 0xCC40CC40u};
+#pragma unroll
+        for (int wi = 0; wi < 2; ++wi)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t x = j < 4 ? words[wi] : words[wi] >> 8;
+                const int jj = j & 3;
+                ka[4 * wi + (j >> 1)][j & 1] =
+                    hfma2_u32(and_or(x, 0x00030003u << (2 * jj), kMagic), mul[jj], add[jj]);
+            }
+    } else if constexpr (BITS == 3) {
+        const uint32_t* p = reinterpret_cast<const uint32_t*>(row + 12 * t);
+        const uint32_t W0 = p[0], W1 = p[1], W2 = p[2];
+        const uint32_t G[4] = {W0, prmt(W0, W1, 0x6543u), prmt(W1, W2, 0x5432u), W2 >> 8};
+        constexpr uint32_t mul[3] = {0x3C003C00u, 0x30003000u, 0x24002400u};
+        constexpr uint32_t add[3] = {0xE403E403u, 0xD818D818u, 0xCCC0CCC0u};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t sel = bitsel(G[q], G[q] << 4, 0x0000FFFFu);
+            const uint32_t sel3 = bitsel(G[q] >> 3, G[q] << 1, 0x0000FFFFu);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t pr = k < 3 ? and_or(sel, 0x00070007u << (3 * k), kMagic)
+                                          : and_or(sel3, 0x01C001C0u, kMagic);
+                const int kk = k < 3 ? k : 2;
+                ka[2 * q + (k >> 1)][k & 1] = hfma2_u32(pr, mul[kk], add[kk]);
+            }
+        }
+    } else {  // bf16: dims 32t .. 32t+31, adjacent pairs as stored
+#pragma unroll
+        for (int w4 = 0; w4 < 4; ++w4) {
+            const uint4 x = *reinterpret_cast<const uint4*>(row + 64 * t + 16 * w4);
+            ka[2 * w4][0] = x.x;
+            ka[2 * w4][1] = x.y;
+            ka[2 * w4 + 1][0] = x.z;
+            ka[2 * w4 + 1][1] = x.w;
+        }
+    }
+}
+
+// ----------------------------------------------------------- V unpackers
+// va[mt][i]: A-fragment of V^T for m-tile mt (rows = dims 16g + 2mt and
+// 16g + 2mt + 1), k = tokens {t, t+4} (i = 0, 1) and {t+8, t+12} (i = 2, 3).
+template <int BITS>
+__device__ __forceinline__ void unpack_v(const uint8_t* codes, int g, int t, uint32_t va[8][4])
+{
+    constexpr int CB = Fmt<BITS>::CB;
+    const uint8_t* r0 = codes + (t + 0) * CB;
+    const uint8_t* r1 = codes + (t + 4) * CB;
+    const uint8_t* r2 = codes + (t + 8) * CB;
+    const uint8_t* r3 = codes + (t + 12) * CB;
+    if constexpr (BITS == 4) {
+        const uint2 X[4] = {*reinterpret_cast<const uint2*>(r0 + 8 * g),
+                            *reinterpret_cast<const uint2*>(r1 + 8 * g),
+                            *reinterpret_cast<const uint2*>(r2 + 8 * g),
+                            *reinterpret_cast<const uint2*>(r3 + 8 * g)};
+#pragma unroll
+        for (int p = 0; p < 2; ++p)
+#pragma unroll
+            for (int hw = 0; hw < 2; ++hw) {
+                const uint32_t xw = hw ? X[2 * p].y : X[2 * p].x;
+                const uint32_t yw = hw ? X[2 * p + 1].y : X[2 * p + 1].x;
+#pragma unroll
+                for (int xs = 0; xs < 2; ++xs) {
+                    const uint32_t xx = prmt(xw, yw, xs ? 0x7632u : 0x5410u);
+                    const uint32_t x8 = xx >> 8;
+                    const uint32_t d[4] = {
+                        hfma2_u32(and_or(xx, 0x000F000Fu, kMagic), 0x3C003C00u, 0xE407E407u),
+                        hfma2_u32(and_or(xx, 0x00F000F0u, kMagic), 0x2C002C00u, 0xD470D470u),
+                        hfma2_u32(and_or(x8, 0x000F000Fu, kMagic), 0x3C003C00u, 0xE407E407u),
+                        hfma2_u32(and_or(x8, 0x00F000F0u, kMagic), 0x2C002C00u, 0xD470D470u)};
+#pragma unroll
+                    for (int n = 0; n < 4; ++n) {
+                        const int dl = 8 * hw + 4 * xs + n;   // dim 16g + dl
+                        va[dl >> 1][(dl & 1) + 2 * p] = d[n];
+                    }
+                }
+            }
+    } else if constexpr (BITS == 8) {
+        const uint4 X[4] = {*reinterpret_cast<const uint4*>(r0 + 16 * g),
+                            *reinterpret_cast<const uint4*>(r1 + 16 * g),
+                            *reinterpret_cast<const uint4*>(r2 + 16 * g),
+                            *reinterpret_cast<const uint4*>(r3 + 16 * g)};
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const uint32_t xa[4] = {X[2 * p].x, X[2 * p].y, X[2 * p].z, X[2 * p].w};
+            const uint32_t ya[4] = {X[2 * p + 1].x, X[2 * p + 1].y, X[2 * p + 1].z, X[2 * p + 1].w};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const uint32_t t1 = prmt(xa[w], ya[w], 0x5410u);
+                const uint32_t t2 = prmt(xa[w], ya[w], 0x7632u);
+                const uint32_t d[4] = {
+                    hfma2_u32(prmt(t1, 0x64646464u, 0x4240u), 0x3C003C00u, 0xE47FE47Fu),
+                    hfma2_u32(prmt(t1, 0x64646464u, 0x4341u), 0x3C003C00u, 0xE47FE47Fu),
+                    hfma2_u32(prmt(t2, 0x64646464u, 0x4240u), 0x3C003C00u, 0xE47FE47Fu),
+                    hfma2_u32(prmt(t2, 0x64646464u, 0x4341u), 0x3C003C00u, 0xE47FE47Fu)};
+#pragma unroll
+                for (int n = 0; n < 4; ++n) {
+                    const int dl = 4 * w + n;
+                    va[dl >> 1][(dl & 1) + 2 * p] = d[n];
+                }
+            }
+        }
+    } else if constexpr (BITS == 2) {
+        const uint32_t X[4] = {*reinterpret_cast<const uint32_t*>(r0 + 4 * g),
+                               *reinterpret_cast<const uint32_t*>(r1 + 4 * g),
+                               *reinterpret_cast<const uint32_t*>(r2 + 4 * g),
+                               *reinterpret_cast<const uint32_t*>(r3 + 4 * g)};
+        constexpr uint32_t mul[4] = {0x3C003C00u, 0x34003400u, 0x2C002C00u, 0x24002400u};
+        constexpr uint32_t add[4] = {0xE401E401u, 0xDC04DC04u, 0xD410D410u, 0xCC40CC40u};
+#pragma unroll
+        for (int p = 0; p < 2; ++p)
+#pragma unroll
+            for (int xi = 0; xi < 2; ++xi) {
+                const uint32_t xx = prmt(X[2 * p], X[2 * p + 1], xi ? 0x7632u : 0x5410u);
+                const uint32_t x8 = xx >> 8;
+#pragma unroll
+                for (int n = 0; n < 8; ++n) {
+                    const int jj = n & 3;
+                    const uint32_t v = hfma2_u32(
+                        and_or(n < 4 ? xx : x8, 0x00030003u << (2 * jj), kMagic), mul[jj], add[jj]);
+                    const int dl = 8 * xi + n;
+                    va[dl >> 1][(dl & 1) + 2 * p] = v;
+                }
+            }
+    } else if constexpr (BITS == 3) {
+        // 48 bits per token at bit 48g; read two aligned words and shift
+        const int byte0 = 6 * g;
+        const int base = byte0 & ~3;
+        const int sh = (byte0 & 3) * 8;
+        uint64_t bits[4];
+        const uint8_t* rows[4] = {r0, r1, r2, r3};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(rows[i] + base);
+            const uint64_t v64 = ((uint64_t)w[1] << 32) | w[0];
+            bits[i] = v64 >> sh;
+        }
+        constexpr uint32_t mul[3] = {0x3C003C00u, 0x30003000u, 0x24002400u};
+        constexpr uint32_t add[3] = {0xE403E403u, 0xD818D818u, 0xCCC0CCC0u};
+#pragma unroll
+        for (int p = 0; p < 2; ++p)
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const uint32_t a12 = (uint32_t)(bits[2 * p] >> (12 * m)) & 0xFFFu;
+                const uint32_t b12 = (uint32_t)(bits[2 * p + 1] >> (12 * m)) & 0xFFFu;
+                const uint32_t xy = a12 | (b12 << 16);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t pr = k < 3 ? and_or(xy, 0x00070007u << (3 * k), kMagic)
+                                              : and_or(xy >> 3, 0x01C001C0u, kMagic);
+                    const int kk = k < 3 ? k : 2;
+                    const int dl = 4 * m + k;
+                    va[dl >> 1][(dl & 1) + 2 * p] = hfma2_u32(pr, mul[kk], add[kk]);
+                }
+            }
+    } else {  // bf16
+        uint4 X[4][2];
+        const uint8_t* rows[4] = {r0, r1, r2, r3};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            X[i][0] = *reinterpret_cast<const uint4*>(rows[i] + 32 * g);
+            X[i][1] = *reinterpret_cast<const uint4*>(rows[i] + 32 * g + 16);
+        }
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const uint32_t xa[8] = {X[2 * p][0].x, X[2 * p][0].y, X[2 * p][0].z, X[2 * p][0].w,
+                                    X[2 * p][1].x, X[2 * p][1].y, X[2 * p][1].z, X[2 * p][1].w};
+            const uint32_t ya[8] = {X[2 * p + 1][0].x, X[2 * p + 1][0].y, X[2 * p + 1][0].z,
+                                    X[2 * p + 1][0].w, X[2 * p + 1][1].x, X[2 * p + 1][1].y,
+                                    X[2 * p + 1][1].z, X[2 * p + 1][1].w};
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                va[mt][2 * p] = prmt(xa[mt], ya[mt], 0x5410u);
+                va[mt][2 * p + 1] = prmt(xa[mt], ya[mt], 0x7632u);
+            }
+        }
+    }
+}
+
+template <int BITS>
+__device__ __forceinline__ void issue_tile(uint8_t* dst, uint64_t* bar, const DecodeArgs& a,
+                                           int page, int kvh, int sub)
+{
+    using F = Fmt<BITS>;
+    const int64_t blk = ((int64_t)page * a.num_kv_heads + kvh) * a.block_bytes;
+    const uint8_t* kb = a.kp + blk;
+    const uint8_t* vb = a.vp + blk;
+    mbar_arrive_expect_tx(bar, F::kStageBytes);
+    bulk_g2s(dst, kb + sub * F::kTileCodes, F::kTileCodes, bar);
+    bulk_g2s(dst + F::kVOff, vb + sub * F::kTileCodes, F::kTileCodes, bar);
+    if constexpr (F::kTurbo) {
+        const int64_t so = (int64_t)a.page_size * F::CB + 64 * sub;
+        bulk_g2s(dst + F::kTileCodes, kb + so, 64, bar);
+        bulk_g2s(dst + F::kVOff + F::kTileCodes, vb + so, 64, bar);
+    }
+}
+
+__device__ __forceinline__ void fwht128_lane(float x[4], int lane)
+{
+    float a0 = x[0] + x[1], a1 = x[0] - x[1], a2 = x[2] + x[3], a3 = x[2] - x[3];
+    x[0] = a0 + a2;
+    x[2] = a0 - a2;
+    x[1] = a1 + a3;
+    x[3] = a1 - a3;
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+        const bool upper = (lane & m) != 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float p = __shfl_xor_sync(kFull, x[e], m);
+            x[e] = upper ? p - x[e] : x[e] + p;
+        }
+    }
+}
+
+__device__ __forceinline__ float pow2i(int e)  // 2^e for -126 <= e <= 127
+{
+    e = max(-126, min(127, e));
+    return __uint_as_float((uint32_t)(e + 127) << 23);
+}
+
+template <int BITS, int NT>
+__global__ void __launch_bounds__(kThreads)
+k_decode(const DecodeArgs a)
+{
+    using F = Fmt<BITS>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    float* sQ = reinterpret_cast<float*>(smem);                      // [8][128]
+    float* sRowFac = sQ + kRowsPerCta * kHeadDim;                    // [8]
+    int* sFlag = reinterpret_cast<int*>(sRowFac + 16);               // [4]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 4352 - 128); // [4][kMaxStages]
+    uint8_t* ring = smem + 4352;
+
+    const int split = blockIdx.x;
+    const int b = blockIdx.z;
+    const int kvh = blockIdx.y / a.R;
+    const int rg = blockIdx.y - kvh * a.R;
+    const int seq_len = a.seq_lens[b];
+    if (seq_len < a.q_len || seq_len > a.max_seq_len) {
+        if (split == 0 && blockIdx.y == 0 && threadIdx.x == 0)
+            report_error(a.err, TQ_ERR_DEVICE_CHECK, kErrSeqLen);
+        return;
+    }
+    const int nsplit = (seq_len + a.split_tokens - 1) / a.split_tokens;
+    if (split >= nsplit) return;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int tok_begin = split * a.split_tokens;
+    const int tok_end = min(seq_len, tok_begin + a.split_tokens);
+    const int ntiles = (tok_end - tok_begin + 15) >> 4;
+    const int my_tiles = ntiles > warp ? (ntiles - warp + kWarps - 1) / kWarps : 0;
+    const int stages = a.stages;
+    uint64_t* mybar = bars + warp * kMaxStages;
+    uint8_t* myring = ring + warp * stages * F::kStageBytes;
+
+    // physical page of each of my tiles: lane j holds tile j
+    int pid = 0, psub = 0;
+    if (lane < my_tiles) {
+        const int tok = tok_begin + 16 * (warp + kWarps * lane);
+        pid = __ldg(a.page_table + (int64_t)b * a.max_pages + tok / a.page_size);
+        psub = (tok % a.page_size) >> 4;
+        if (pid < 0 || pid >= a.num_pages) {
+            report_error(a.err, TQ_ERR_DEVICE_CHECK, kErrPageRange);
+            pid = 0;
+        }
+    }
+    if (lane == 0) {
+        for (int s = 0; s < stages; ++s) mbar_init(&mybar[s], 1);
+        fence_barrier_init();
+    }
+    if (threadIdx.x == 0) sFlag[0] = 0;
+    __syncwarp();
+    const int first = min(stages, my_tiles);
+    for (int i = 0; i < first; ++i) {
+        const int p = __shfl_sync(kFull, pid, i);
+        const int sb = __shfl_sync(kFull, psub, i);
+        if (lane == 0) issue_tile<BITS>(myring + i * F::kStageBytes, &mybar[i], a, p, kvh, sb);
+    }
+
+    // ---- rotated, scaled query rows of this row group (while tiles load)
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int rr = warp + 4 * k;
+        const int r = rg * kRowsPerCta + rr;
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        if (r < a.G) {
+            const int tq = r / a.group;
+            const int h = kvh * a.group + (r - tq * a.group);
+            const uint2 raw = __ldg(reinterpret_cast<const uint2*>(
+                a.q + (((int64_t)b * a.q_len + tq) * a.num_q_heads + h) * kHeadDim) + lane);
+            x[0] = bf16_bits_to_float(raw.x & 0xffffu);
+            x[1] = bf16_bits_to_float(raw.x >> 16);
+            x[2] = bf16_bits_to_float(raw.y & 0xffffu);
+            x[3] = bf16_bits_to_float(raw.y >> 16);
+        }
+        float fac;
+        if constexpr (F::kTurbo) {
+            fwht128_lane(x, lane);
+            fac = kLog2e / kHeadDim;        // (H q / sqrt d) . y / sqrt d = (H q) . y / d
+        } else {
+            fac = kLog2e * 0.08838834764831845f;  // 1 / sqrt(128)
+        }
+        float amax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            x[e] *= fac;
+            amax = fmaxf(amax, fabsf(x[e]));
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, m));
+        // power-of-two prescale: largest |q'| in [2^12, 2^13) keeps hi and lo
+        // f16 parts normal; the inverse factor is applied to the scores
+        const int ex = amax > 0.f ? max(-100, min(100, ilogbf(amax))) : 0;
+        const float pre = pow2i(12 - ex);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sQ[rr * kHeadDim + 4 * lane + e] = x[e] * pre;
+        if (lane == 0) sRowFac[rr] = pow2i(ex - 12);
+    }
+    __syncthreads();
+
+    // B fragments of the query: column n = g holds row 4nt + (g & 3), hi
+    // part for g < 4, lo part for g >= 4
+    uint32_t qf[NT][8][2];
+    float rowfac[NT][2];
+    int lim[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const float* qrow = sQ + (4 * nt + (g & 3)) * kHeadDim;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+#pragma unroll
+            for (int f = 0; f < 2; ++f) {
+                const float v0 = qrow[qk_dim<BITS>(t, c, f, 0)];
+                const float v1 = qrow[qk_dim<BITS>(t, c, f, 1)];
+                if constexpr (F::kTurbo) {
+                    const float h0 = __half2float(__float2half_rn(v0));
+                    const float h1 = __half2float(__float2half_rn(v1));
+                    qf[nt][c][f] = g < 4 ? pack_half2(v0, v1) : pack_half2(v0 - h0, v1 - h1);
+                } else {
+                    const float h0 = __bfloat162float(__float2bfloat16_rn(v0));
+                    const float h1 = __bfloat162float(__float2bfloat16_rn(v1));
+                    qf[nt][c][f] = g < 4 ? pack_bf162(v0, v1) : pack_bf162(v0 - h0, v1 - h1);
+                }
+            }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int rl = 4 * nt + 2 * (t & 1) + e;
+            const int r = rg * kRowsPerCta + rl;
+            rowfac[nt][e] = sRowFac[rl];
+            lim[nt][e] = r < a.G ? seq_len - a.q_len + r / a.group : -1;
+        }
+    }
+
+    float o[NT][8][4];
+    float m_run[NT][2], l_run[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[nt][mt][i] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            m_run[nt][e] = -CUDART_INF_F;
+            l_run[nt][e] = 0.f;
+        }
+    }
+    int ev = 0;   // running biased fp32 exponent of the V scales (turbo)
+    const float kinv = F::kTurbo ? 1.f / (float)F::L : 1.f;
+
+    int failed_at = -1;
+    for (int i = 0; i < my_tiles; ++i) {
+        const int slot = i % stages;
+        if (!mbar_wait_bounded(&mybar[slot], (uint32_t)((i / stages) & 1), kWaitSpins)) {
+            if (lane == 0) report_error(a.err, TQ_ERR_TIMEOUT, kErrWaitTile);
+            failed_at = i;
+            break;
+        }
+        const uint8_t* st = myring + slot * F::kStageBytes;
+        const int tok0 = tok_begin + 16 * (warp + kWarps * i);
+        const int ra = perm(g), rb = perm(g + 8);
+
+        // ---------------- S = K q'
+        float s[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) s[nt][k] = 0.f;
+        {
+            uint32_t ka[8][2], kb[8][2];
+            unpack_k<BITS>(st + ra * F::CB, t, ka);
+            unpack_k<BITS>(st + rb * F::CB, t, kb);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint32_t afr[4] = {ka[c][0], kb[c][0], ka[c][1], kb[c][1]};
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    if constexpr (F::kTurbo) mma_f16(s[nt], afr, qf[nt][c][0], qf[nt][c][1]);
+                    else mma_bf16(s[nt], afr, qf[nt][c][0], qf[nt][c][1]);
+                }
+            }
+        }
+        // hi + lo columns, then scale to log2 units
+        float ks0 = 1.f, ks1 = 1.f, vs0 = 1.f, vs1 = 1.f;
+        if constexpr (F::kTurbo) {
+            const float* kscale = reinterpret_cast<const float*>(st + F::kTileCodes);
+            const float* vscale = reinterpret_cast<const float*>(st + F::kVOff + F::kTileCodes);
+            ks0 = kscale[ra] * kinv;
+            ks1 = kscale[rb] * kinv;
+            vs0 = vscale[ra] * kinv;
+            vs1 = vscale[rb] * kinv;
+        }
+        const int ja = tok0 + ra, jb = tok0 + rb;
+        // slots past the sequence end were never written: keep their
+        // (arbitrary) scales out of every product
+        if (ja >= seq_len) { ks0 = 0.f; vs0 = 0.f; }
+        if (jb >= seq_len) { ks1 = 0.f; vs1 = 0.f; }
+        float sc[NT][4];
+        bool need = false;
+        int vexp = 0;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float s0 = s[nt][e] + __shfl_xor_sync(kFull, s[nt][e], 2);
+                const float s1 = s[nt][2 + e] + __shfl_xor_sync(kFull, s[nt][2 + e], 2);
+                const bool v0 = ja <= lim[nt][e], v1 = jb <= lim[nt][e];
+                sc[nt][e] = v0 ? s0 * ks0 * rowfac[nt][e] : -CUDART_INF_F;
+                sc[nt][2 + e] = v1 ? s1 * ks1 * rowfac[nt][e] : -CUDART_INF_F;
+                need |= fmaxf(sc[nt][e], sc[nt][2 + e]) > m_run[nt][e] + kLazyThreshold;
+                if constexpr (F::kTurbo) {
+                    if (v0) vexp = max(vexp, (int)((__float_as_uint(vs0) >> 23) & 0xFF));
+                    if (v1) vexp = max(vexp, (int)((__float_as_uint(vs1) >> 23) & 0xFF));
+                }
+            }
+        int ev_new = ev;
+        if constexpr (F::kTurbo) ev_new = max(ev, (int)__reduce_max_sync(kFull, (unsigned)vexp));
+        if (__any_sync(kFull, need) || ev_new != ev) {
+            const float av = F::kTurbo ? pow2i(ev - ev_new) : 1.f;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    float v = fmaxf(sc[nt][e], sc[nt][2 + e]);
+                    v = fmaxf(v, __shfl_xor_sync(kFull, v, 4));
+                    v = fmaxf(v, __shfl_xor_sync(kFull, v, 8));
+                    v = fmaxf(v, __shfl_xor_sync(kFull, v, 16));
+                    const float mn = fmaxf(m_run[nt][e], v);
+                    const float alpha = mn == -CUDART_INF_F ? 1.f : exp2f(m_run[nt][e] - mn);
+                    m_run[nt][e] = mn;
+                    l_run[nt][e] *= alpha;
+                    const float ao = alpha * av;
+#pragma unroll
+                    for (int mt = 0; mt < 8; ++mt) {
+                        o[nt][mt][e] *= ao;
+                        o[nt][mt][2 + e] *= ao;
+                    }
+                }
+            ev = ev_new;
+        }
+        // P' = p * s_v / L * 2^-(ev-127), split into hi (lanes t < 2) and
+        // lo (t >= 2) halves, transposed onto the PV B fragment
+        const float vn = F::kTurbo ? pow2i(127 - ev) : 1.f;
+        const float vn0 = vs0 * vn, vn1 = vs1 * vn;
+        uint32_t pb[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            float pv[4];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float p0 = sc[nt][e] == -CUDART_INF_F ? 0.f : exp2f(sc[nt][e] - m_run[nt][e]);
+                const float p1 = sc[nt][2 + e] == -CUDART_INF_F ? 0.f : exp2f(sc[nt][2 + e] - m_run[nt][e]);
+                l_run[nt][e] += p0 + p1;
+                pv[e] = p0 * vn0;
+                pv[2 + e] = p1 * vn1;
+            }
+            uint32_t top, bot;
+            if constexpr (F::kTurbo) {
+                if (t < 2) {
+                    top = pack_half2(pv[0], pv[1]);
+                    bot = pack_half2(pv[2], pv[3]);
+                } else {
+                    top = pack_half2(pv[0] - __half2float(__float2half_rn(pv[0])),
+                                     pv[1] - __half2float(__float2half_rn(pv[1])));
+                    bot = pack_half2(pv[2] - __half2float(__float2half_rn(pv[2])),
+                                     pv[3] - __half2float(__float2half_rn(pv[3])));
+                }
+            } else {
+                if (t < 2) {
+                    top = pack_bf162(pv[0], pv[1]);
+                    bot = pack_bf162(pv[2], pv[3]);
+                } else {
+                    top = pack_bf162(pv[0] - __bfloat162float(__float2bfloat16_rn(pv[0])),
+                                     pv[1] - __bfloat162float(__float2bfloat16_rn(pv[1])));
+                    bot = pack_bf162(pv[2] - __bfloat162float(__float2bfloat16_rn(pv[2])),
+                                     pv[3] - __bfloat162float(__float2bfloat16_rn(pv[3])));
+                }
+            }
+            pb[nt][0] = movmatrix_trans(top);
+            pb[nt][1] = movmatrix_trans(bot);
+        }
+
+        // ---------------- O^T += V^T P'
+        {
+            uint32_t va[8][4];
+            unpack_v<BITS>(st + F::kVOff, g, t, va);
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    if constexpr (F::kTurbo) mma_f16(o[nt][mt], va[mt], pb[nt][0], pb[nt][1]);
+                    else mma_bf16(o[nt][mt], va[mt], pb[nt][0], pb[nt][1]);
+                }
+        }
+
+        __syncwarp();
+        if (i + stages < my_tiles) {
+            const int p = __shfl_sync(kFull, pid, i + stages);
+            const int sb = __shfl_sync(kFull, psub, i + stages);
+            if (lane == 0)
+                issue_tile<BITS>(myring + slot * F::kStageBytes, &mybar[slot], a, p, kvh, sb);
+        }
+    }
+
+    if (failed_at >= 0) {
+        // drain this warp's copies still in flight (bounded), then give up
+        const int last = min(my_tiles, failed_at + stages);
+        for (int j = failed_at + 1; j < last; ++j)
+            (void)mbar_wait_bounded(&mybar[j % stages], (uint32_t)((j / stages) & 1), kWaitSpins);
+        if (lane == 0) atomicExch(&sFlag[0], 1);
+    }
+
+    // ---- warp partials -> shared memory (the ring is free now)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            float l = l_run[nt][e];
+            l += __shfl_xor_sync(kFull, l, 4);
+            l += __shfl_xor_sync(kFull, l, 8);
+            l += __shfl_xor_sync(kFull, l, 16);
+            l_run[nt][e] = l;
+        }
+    const float vback = F::kTurbo ? pow2i(ev - 127) : 1.f;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                o[nt][mt][i] = (o[nt][mt][i] + __shfl_xor_sync(kFull, o[nt][mt][i], 2)) * vback;
+
+    __syncthreads();  // every warp is done with its ring
+    float* sO = reinterpret_cast<float*>(ring);                          // [4][8][128]
+    float* sM = sO + kWarps * kRowsPerCta * kHeadDim;                    // [4][8]
+    float* sL = sM + kWarps * kRowsPerCta;                               // [4][8]
+    if (t < 2) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int rl = 4 * nt + 2 * t + e;
+                float* dst = sO + (warp * kRowsPerCta + rl) * kHeadDim + 16 * g;
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {
+                    dst[2 * mt] = o[nt][mt][e];
+                    dst[2 * mt + 1] = o[nt][mt][2 + e];
+                }
+                if (g == 0) {
+                    sM[warp * kRowsPerCta + rl] = m_run[nt][e];
+                    sL[warp * kRowsPerCta + rl] = l_run[nt][e];
+                }
+            }
+    }
+    __syncthreads();
+    if (sFlag[0]) return;
+
+    // ---- merge the 4 warps; warp w takes rows w and w + 4
+    const int nrows = min(kRowsPerCta, min(4 * NT, a.G - rg * kRowsPerCta));
+    const int64_t unit = ((int64_t)b * gridDim.y + blockIdx.y);        // (seq, kvh, rg)
+    const int64_t part = unit * a.max_splits + split;
+    const float rs = 0.08838834764831845f;                             // 1 / sqrt(128)
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int rr = warp + 4 * k;
+        if (rr >= nrows) continue;
+        float M = -CUDART_INF_F;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sM[w * kRowsPerCta + rr]);
+        float Lsum = 0.f;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            const float mw = sM[w * kRowsPerCta + rr];
+            const float sc = mw == -CUDART_INF_F ? 0.f : exp2f(mw - M);
+            Lsum += sc * sL[w * kRowsPerCta + rr];
+            const float4 v = *reinterpret_cast<const float4*>(
+                sO + (w * kRowsPerCta + rr) * kHeadDim + 4 * lane);
+            acc[0] += sc * v.x;
+            acc[1] += sc * v.y;
+            acc[2] += sc * v.z;
+            acc[3] += sc * v.w;
+        }
+        const int r = rg * kRowsPerCta + rr;
+        const int tq = r / a.group;
+        const int h = kvh * a.group + (r - tq * a.group);
+        if (nsplit == 1) {
+            const float inv = 1.f / Lsum;
+            float x[4] = {acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv};
+            if constexpr (F::kTurbo) {
+                fwht128_lane(x, lane);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) x[e] *= rs;
+            }
+            *reinterpret_cast<float4*>(a.out + (((int64_t)b * a.q_len + tq) * a.num_q_heads + h) *
+                                                   kHeadDim + 4 * lane) =
+                make_float4(x[0], x[1], x[2], x[3]);
+        } else {
+            *reinterpret_cast<float4*>(a.ws_o + (part * kRowsPerCta + rr) * kHeadDim + 4 * lane) =
+                make_float4(acc[0], acc[1], acc[2], acc[3]);
+            if (lane == 0) a.ws_ml[part * kRowsPerCta + rr] = make_float2(M, Lsum);
+        }
+    }
+    if (nsplit == 1) return;
+
+    // ---- last CTA of this (seq, kv head, row group) merges every split
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned old = atomicInc(a.ws_cnt + unit, (unsigned)(nsplit - 1));
+        sFlag[1] = old == (unsigned)(nsplit - 1);
+    }
+    __syncthreads();
+    if (!sFlag[1]) return;
+    __threadfence();
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int rr = warp + 4 * k;
+        if (rr >= nrows) continue;
+        const int64_t base = unit * a.max_splits;
+        float M = -CUDART_INF_F;
+        for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, __ldcg(a.ws_ml + (base + sp) * kRowsPerCta + rr).x);
+        float Lsum = 0.f;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int sp = 0; sp < nsplit; ++sp) {
+            const float2 ml = __ldcg(a.ws_ml + (base + sp) * kRowsPerCta + rr);
+            const float sc = ml.x == -CUDART_INF_F ? 0.f : exp2f(ml.x - M);
+            Lsum += sc * ml.y;
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(
+                a.ws_o + ((base + sp) * kRowsPerCta + rr) * kHeadDim) + lane);
+            acc[0] += sc * v.x;
+            acc[1] += sc * v.y;
+            acc[2] += sc * v.z;
+            acc[3] += sc * v.w;
+        }
+        const float inv = 1.f / Lsum;
+        float x[4] = {acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv};
+        if constexpr (F::kTurbo) {
+            fwht128_lane(x, lane);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) x[e] *= rs;
+        }
+        const int r = rg * kRowsPerCta + rr;
+        const int tq = r / a.group;
+        const int h = kvh * a.group + (r - tq * a.group);
+        *reinterpret_cast<float4*>(a.out + (((int64_t)b * a.q_len + tq) * a.num_q_heads + h) *
+                                               kHeadDim + 4 * lane) =
+            make_float4(x[0], x[1], x[2], x[3]);
+    }
+}
+
+template <int BITS>
+int stages_for()
+{
+    const int s = 9216 / Fmt<BITS>::kStageBytes;
+    return s < 2 ? 2 : (s > kMaxStages ? kMaxStages : s);
+}
+
+template <int BITS>
+size_t smem_for(int stages)
+{
+    const size_t ring = (size_t)kWarps * stages * Fmt<BITS>::kStageBytes;
+    const size_t merge = (size_t)kWarps * kRowsPerCta * (kHeadDim + 2) * sizeof(float);
+    return 4352 + (ring > merge ? ring : merge);
+}
+
+template <int BITS, int NT>
+cudaError_t launch_one(DecodeArgs a, dim3 grid, cudaStream_t stream)
+{
+    a.stages = stages_for<BITS>();
+    const size_t smem = smem_for<BITS>(a.stages);
+    static int configured_device_mask = 0;   // one bit per device ordinal < 31
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 31 || !(configured_device_mask & (1 << dev))) {
+        e = cudaFuncSetAttribute(k_decode<BITS, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+        if (e != cudaSuccess) return e;
+        if (dev < 31) configured_device_mask |= 1 << dev;
+    }
+    k_decode<BITS, NT><<<grid, kThreads, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int decode_split_tokens(int page_size) { return page_size >= 64 ? 1024 : 512; }
+
+int decode_row_groups(int G) { return (G + kRowsPerCta - 1) / kRowsPerCta; }
+
+// Workspace: [counters (256-byte aligned)][m,l partials][O partials]
+size_t decode_workspace_bytes(int batch, int num_kv_heads, int G, int max_seq_len, int page_size)
+{
+    const int st = decode_split_tokens(page_size);
+    const int64_t max_splits = (max_seq_len + st - 1) / st;
+    if (max_splits <= 1) return 0;
+    const int64_t units = (int64_t)batch * num_kv_heads * decode_row_groups(G);
+    const int64_t cnt = ((units * 4 + 255) / 256) * 256;
+    const int64_t ml = ((units * max_splits * kRowsPerCta * 8 + 255) / 256) * 256;
+    const int64_t ob = units * max_splits * kRowsPerCta * kHeadDim * 4;
+    return (size_t)(cnt + ml + ob);
+}
+
+cudaError_t launch_decode(const void* q, const tq_cache& c, int64_t block_bytes,
+                          const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                          int batch, int q_len, int num_q_heads, int max_seq_len, float* out,
+                          void* workspace, cudaStream_t stream)
+{
+    DecodeArgs a{};
+    a.q = static_cast<const uint16_t*>(q);
+    a.kp = static_cast<const uint8_t*>(c.k_pages);
+    a.vp = static_cast<const uint8_t*>(c.v_pages);
+    a.page_table = page_table;
+    a.seq_lens = seq_lens;
+    a.out = out;
+    a.err = c.dev_error;
+    a.block_bytes = block_bytes;
+    a.max_pages = max_pages;
+    a.num_pages = c.num_pages;
+    a.num_kv_heads = c.num_kv_heads;
+    a.num_q_heads = num_q_heads;
+    a.group = num_q_heads / c.num_kv_heads;
+    a.q_len = q_len;
+    a.G = q_len * a.group;
+    a.R = decode_row_groups(a.G);
+    a.page_size = c.page_size;
+    a.split_tokens = decode_split_tokens(c.page_size);
+    a.max_splits = (max_seq_len + a.split_tokens - 1) / a.split_tokens;
+    a.max_seq_len = max_seq_len;
+    if (a.max_splits > 1) {
+        const int64_t units = (int64_t)batch * c.num_kv_heads * a.R;
+        const int64_t cnt = ((units * 4 + 255) / 256) * 256;
+        const int64_t ml = ((units * a.max_splits * kRowsPerCta * 8 + 255) / 256) * 256;
+        uint8_t* w = static_cast<uint8_t*>(workspace);
+        a.ws_cnt = reinterpret_cast<uint32_t*>(w);
+        a.ws_ml = reinterpret_cast<float2*>(w + cnt);
+        a.ws_o = reinterpret_cast<float*>(w + cnt + ml);
+    }
+    const dim3 grid((unsigned)a.max_splits, (unsigned)(c.num_kv_heads * a.R), (unsigned)batch);
+    const bool two = (a.G > 4);   // more than 4 rows in a row group
+#define TQ_DEC(B)                                                                      \
+    return two ? launch_one<B, 2>(a, grid, stream) : launch_one<B, 1>(a, grid, stream)
+    switch (c.format) {
+    case 2: TQ_DEC(2);
+    case 3: TQ_DEC(3);
+    case 4: TQ_DEC(4);
+    case 8: TQ_DEC(8);
+    case 16: TQ_DEC(16);
+    default: return cudaErrorInvalidValue;
+    }
+#undef TQ_DEC
+}
+
+}  // namespace tq

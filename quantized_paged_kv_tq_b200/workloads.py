@@ -271,7 +271,9 @@ def custom(name="custom", batch=2, num_q_heads=8, num_kv_heads=2, page_size=16,
            q_len=1, seq_lens=(40, 17), fmt=4, seed=123, k_outliers=2,
            v_outliers=1, permute_pages=True, shared_prefix_seqs=0,
            shared_prefix_tokens=0, k_dist="normal") -> Workload:
-    """A small workload of arbitrary shape for edge-case tests."""
+    """A small workload of arbitrary shape for edge-case tests (the batch is
+    len(seq_lens))."""
+    batch = len(seq_lens)
     w = Workload(name, batch, num_q_heads, num_kv_heads, page_size, q_len,
                  (fmt,), seed, k_dist=k_dist, k_outliers=k_outliers,
                  v_outliers=v_outliers, permute_pages=permute_pages,

@@ -1,0 +1,139 @@
+"""The C ABI on the host (no GPU): symbols, sizes, status codes.
+
+Every call here fails host validation or is a documented no-op, so nothing
+reaches the CUDA runtime."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+from quantized_paged_kv_tq_b200 import build as tqbuild
+
+tqbuild.build()
+from quantized_paged_kv_tq_b200 import tq  # noqa: E402
+
+
+def header_functions():
+    with open(os.path.join(ROOT, "include", "tq.h")) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_and_binding_agree():
+    assert header_functions() == sorted(tq.SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(tq.LIB_PATH)
+    for name in header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_abi_version_and_strings():
+    assert tq.abi_version() == 1
+    for s in range(7):
+        assert tq.status_string(s).startswith("TQ_")
+    assert tq.status_string(99) == "TQ_ERR_UNKNOWN"
+
+
+def test_block_bytes():
+    # page of 16 tokens: d*b/8 code bytes + a 4-byte scale per token
+    assert tq.tq_page_block_bytes(tq.TQ_TURBO4, 128, 16) == 16 * 68
+    assert tq.tq_page_block_bytes(tq.TQ_TURBO3, 128, 16) == 16 * 52
+    assert tq.tq_page_block_bytes(tq.TQ_TURBO8, 128, 16) == 16 * 132
+    assert tq.tq_page_block_bytes(tq.TQ_TURBO2, 128, 64) == 64 * 36
+    assert tq.tq_page_block_bytes(tq.TQ_BF16, 128, 16) == 16 * 256
+    assert tq.tq_page_block_bytes(tq.TQ_TURBO4, 64, 16) == 0
+    assert tq.tq_page_block_bytes(tq.TQ_TURBO4, 128, 24) == 0
+    assert tq.tq_page_block_bytes(5, 128, 16) == 0
+    for fmt in tq.FORMATS:
+        for P in (16, 32, 64):
+            assert tq.tq_page_block_bytes(fmt, 128, P) % 16 == 0
+
+
+FAKE = 0x10000  # never dereferenced: every call below stops in host checks
+
+
+def desc(fmt=4, d=128, H=8, P=16, pages=10, kp=FAKE, vp=FAKE, err=None):
+    return tq.tq_cache(fmt, d, H, P, pages, kp, vp, err)
+
+
+def qa(c, k=FAKE, v=FAKE, s=FAKE, n=4, bits=None):
+    return tq.lib().tq_quantize_append(k, v, s, n, c.format if bits is None else bits,
+                                       ctypes.byref(c), None)
+
+
+def test_quantize_append_validation():
+    I, U = tq.TQ_ERR_INVALID_ARG, tq.TQ_ERR_UNSUPPORTED
+    assert tq.lib().tq_quantize_append(FAKE, FAKE, FAKE, 4, 4, None, None) == I
+    assert qa(desc(fmt=16)) == I                      # bf16 cache
+    assert qa(desc(fmt=5)) == I                       # unknown format
+    assert qa(desc(), bits=3) == I                    # bits != cache format
+    assert qa(desc(d=64)) == U
+    assert qa(desc(P=24)) == U
+    assert qa(desc(H=0)) == I
+    assert qa(desc(pages=0)) == I
+    assert qa(desc(kp=None)) == I
+    assert qa(desc(kp=FAKE + 8)) == I                 # 16-byte alignment
+    assert qa(desc(), k=None) == I
+    assert qa(desc(), v=FAKE + 2) == I
+    assert qa(desc(), s=FAKE + 4) == I
+    assert qa(desc(), n=-1) == I
+    assert qa(desc(), n=0) == tq.TQ_OK                # no-op, nothing launched
+    assert tq.lib().tq_append_bf16(FAKE, FAKE, FAKE, 4, ctypes.byref(desc(fmt=4)), None) == I
+    assert tq.lib().tq_append_bf16(FAKE, FAKE, FAKE, 0, ctypes.byref(desc(fmt=16)), None) == 0
+
+
+def dec(c, q=FAKE, pt=FAKE, maxp=512, sl=FAKE, B=8, q_len=1, Hq=32, max_len=4096, out=FAKE,
+        ws=FAKE, ws_n=1 << 30, bf16=False):
+    fn = tq.lib().tq_paged_decode_bf16 if bf16 else tq.lib().tq_paged_decode
+    return fn(q, ctypes.byref(c), pt, maxp, sl, B, q_len, Hq, max_len, out, ws, ws_n, None)
+
+
+def test_decode_validation():
+    I, U, W = tq.TQ_ERR_INVALID_ARG, tq.TQ_ERR_UNSUPPORTED, tq.TQ_ERR_WORKSPACE
+    c = desc()
+    assert dec(desc(fmt=16)) == I                     # turbo call on a bf16 cache
+    assert dec(c, bf16=True) == I                     # bf16 call on a turbo cache
+    assert dec(c, Hq=30) == I                         # not a multiple of kv heads
+    assert dec(c, q_len=0) == I
+    assert dec(c, max_len=0) == I
+    assert dec(c, maxp=255) == I                      # too few page-table columns
+    assert dec(c, q_len=17, Hq=32) == U               # 68 rows per kv head > 64
+    assert dec(c, B=70000) == U
+    assert dec(c, q=FAKE + 4) == I
+    assert dec(c, out=FAKE + 8) == I
+    assert dec(c, pt=None) == I
+    assert dec(c, ws=None, ws_n=0) == W
+    assert dec(c, ws_n=1024) == W
+    assert dec(c, B=0) == tq.TQ_OK                    # empty batch: no-op
+    assert dec(c, max_len=4, q_len=8) == I            # max_seq_len < q_len
+
+
+def test_workspace_size():
+    c = desc()
+    ws = tq.lib().tq_decode_workspace_size
+    # one split (<= 512 tokens with 16-token pages): no workspace
+    assert ws(8, 1, 32, 512, ctypes.byref(c)) == 0
+    n = ws(8, 1, 32, 4096, ctypes.byref(c))
+    # 8 splits x 64 (seq, kv head) units x 8 rows x (128 + 2) floats + counters
+    assert n >= 8 * 64 * 8 * 130 * 4 and n < 8 * 64 * 8 * 130 * 4 + 4096
+    assert ws(8, 1, 30, 4096, ctypes.byref(c)) == 0   # invalid
+    c64 = desc(P=64)
+    assert ws(4, 1, 40, 131072, ctypes.byref(c64)) >= 4 * 8 * 128 * 8 * 130 * 4
+
+
+def test_hbm_probe_validation():
+    assert tq.lib().tq_hbm_copy(FAKE, FAKE, 0, None) == 0
+    assert tq.lib().tq_hbm_copy(FAKE, FAKE, 24, None) == tq.TQ_ERR_INVALID_ARG
+    assert tq.lib().tq_hbm_read(FAKE + 4, 32, FAKE, None) == tq.TQ_ERR_INVALID_ARG
+
+
+def test_read_device_error_without_word():
+    code = ctypes.c_uint32(7)
+    assert tq.lib().tq_read_device_error(ctypes.byref(desc(err=None)), ctypes.byref(code), 1,
+                                         None) == 0
+    assert code.value == 0

@@ -1,0 +1,269 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Codes and scales must be bit-exact; attention outputs within max-abs 2e-3
+and relative-L2 1e-3 of the oracle's fp64 result on the same dequantised
+cache.  Small workloads are compared element by element everywhere; the
+full-size workloads on sampled slots and sampled sequences (the oracle
+rebuilds those sequences' caches itself from the generator's values)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import (check_close, dev, dev_bf16, gpu_decode, gpu_fill, gpu_rows,
+                         oracle_decode, oracle_pools, oracle_rows)
+from quantized_paged_kv_tq_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from quantized_paged_kv_tq_b200 import build as _b
+    _b.build()
+    from quantized_paged_kv_tq_b200 import tq
+
+TURBO = (2, 3, 4, 8)
+
+
+def small(fmt, **kw):
+    base = dict(batch=3, num_q_heads=8, num_kv_heads=2, page_size=16, q_len=1,
+                seq_lens=(1300, 37, 513), fmt=fmt, seed=11 + fmt)
+    base.update(kw)
+    return W.custom(**base)
+
+
+# ------------------------------------------------------------ quantiser
+@pytest.mark.parametrize("fmt", TURBO)
+@pytest.mark.parametrize("P", [16, 32, 64])
+def test_quantize_append_bit_exact_small(fmt, P):
+    """Every byte of both pools equals the oracle's (ragged last pages,
+    permuted pages, outlier channels)."""
+    w = small(fmt, page_size=P, seq_lens=(300, 37, 129))
+    cache = gpu_fill(w, fmt)
+    kp, vp = oracle_pools(fmt, w.num_pages, w)
+    for slots, k, v in w.iter_fill():
+        oracle.quantize_append(k, v, slots, fmt, P, kp, vp)
+    assert np.array_equal(cache.k_pages.cpu().numpy(), kp)
+    assert np.array_equal(cache.v_pages.cpu().numpy(), vp)
+    assert cache.read_error() == 0
+
+
+@pytest.mark.parametrize("fmt", TURBO)
+def test_quantize_special_vectors(fmt):
+    """All-zero rows (s = 0), +-powers of two, e_0, constant rows, huge and
+    tiny magnitudes, and slot -1 (skipped)."""
+    rng = np.random.default_rng(fmt)
+    rows = [np.zeros(128, np.float32), np.full(128, 3.0, np.float32), np.eye(128)[0],
+            -np.eye(128)[5] * 1024, rng.standard_normal(128) * 1e30,
+            rng.standard_normal(128) * 1e-30, rng.standard_normal(128) * 2.0 ** 100,
+            np.where(np.arange(128) % 2 == 0, 0.5, -0.5)]
+    n = len(rows)
+    x = np.stack(rows).astype(np.float32)
+    k = W.f32_to_bf16_bits(np.repeat(x[:, None], 2, 1))
+    v = W.f32_to_bf16_bits(np.repeat(-x[:, None], 2, 1))
+    slots = np.arange(n, dtype=np.int64) * 3
+    slots[2] = -1
+    from quantized_paged_kv_tq_b200 import tq as T
+    cache = T.Cache(fmt, 2, 2, 16)
+    T.tq_quantize_append(dev_bf16(k), dev_bf16(v), dev(slots), fmt, cache)
+    torch.cuda.synchronize()
+    kp, vp = oracle_pools(fmt, 2, W.custom(num_kv_heads=2, page_size=16))
+    oracle.quantize_append(k, v, slots, fmt, 16, kp, vp)
+    assert np.array_equal(cache.k_pages.cpu().numpy(), kp)
+    assert np.array_equal(cache.v_pages.cpu().numpy(), vp)
+
+
+@pytest.mark.parametrize("name,fmt", [("tiny", 4), ("batch8", 4), ("cbatch64", 3),
+                                      ("cbatch64", 8), ("target64x8k", 4),
+                                      ("long128k", 4), ("long128k", 2),
+                                      ("specverify", 4)])
+def test_quantize_full_size_sampled(name, fmt):
+    w = W.make(name)
+    cache = gpu_fill(w, fmt)
+    slots = w.fill_slots()
+    pick = np.sort(np.random.default_rng(5).choice(len(slots), min(1500, len(slots)),
+                                                   replace=False))
+    s = slots[pick]
+    got = gpu_rows(cache, s, w.page_size, fmt)
+    ref = oracle_rows(w, s, fmt)
+    for a, b in zip(got, ref):
+        assert np.array_equal(a.view(np.uint8), b.view(np.uint8))
+    assert cache.read_error() == 0
+
+
+# ---------------------------------------------------------------- decode
+@pytest.mark.parametrize("fmt", TURBO + (16,))
+@pytest.mark.parametrize("q_len,Hq,Hkv", [(1, 8, 2), (1, 10, 2), (4, 8, 2), (3, 6, 1),
+                                          (1, 16, 1), (8, 64, 8)])
+def test_decode_small(fmt, q_len, Hq, Hkv):
+    """Ragged lengths (1300 = 2 splits + tail, 37 < one tile, 513 = one
+    token past a split), 1-8 query rows per kv head up to 16 and 64."""
+    w = small(fmt, q_len=q_len, num_q_heads=Hq, num_kv_heads=Hkv,
+              seq_lens=(1300, 37 + q_len, 513))
+    cache = gpu_fill(w, fmt)
+    got = gpu_decode(w, fmt, cache)
+    ref = oracle_decode(w, fmt, np.arange(w.batch))
+    check_close(got, ref, f"fmt {fmt} q_len {q_len} {Hq}/{Hkv}")
+    assert cache.read_error() == 0
+
+
+@pytest.mark.parametrize("fmt", (4, 2))
+def test_decode_page64(fmt):
+    w = small(fmt, page_size=64, seq_lens=(2500, 64, 1025), num_q_heads=10)
+    cache = gpu_fill(w, fmt)
+    check_close(gpu_decode(w, fmt, cache), oracle_decode(w, fmt, np.arange(w.batch)))
+
+
+CONFIG_RUNS = [("tiny", 4, None), ("batch8", 4, (0, 5)), ("cbatch64", 3, "minmax"),
+               ("cbatch64", 8, "minmax"), ("cbatch64", 16, "minmax"),
+               ("target64x8k", 4, (0, 63)), ("long128k", 4, (2,)), ("long128k", 2, (1,)),
+               ("specverify", 4, (0, 7, 20))]
+
+
+@pytest.mark.parametrize("name,fmt,seqs", CONFIG_RUNS)
+def test_decode_configs(name, fmt, seqs):
+    """Every configuration at full size; the oracle checks sampled sequences
+    (all of them for the tiny one) and every output must be finite."""
+    w = W.make(name)
+    cache = gpu_fill(w, fmt)
+    got = gpu_decode(w, fmt, cache)
+    assert np.all(np.isfinite(got))
+    if seqs is None:
+        seqs = np.arange(w.batch)
+    elif seqs == "minmax":
+        seqs = (int(np.argmin(w.seq_lens)), int(np.argmax(w.seq_lens)), 17)
+    seqs = np.asarray(seqs)
+    ref = oracle_decode(w, fmt, seqs)
+    check_close(got[seqs], ref, f"{name} fmt {fmt}")
+    assert cache.read_error() == 0
+
+
+# ------------------------------------------------------------ properties
+@pytest.mark.parametrize("fmt", (4, 16))
+def test_batch_invariance(fmt):
+    """A sequence's output is bit-identical alone and inside a batch."""
+    w = small(fmt, seq_lens=(1300, 37, 513, 2049), batch=4)
+    cache = gpu_fill(w, fmt)
+    full = gpu_decode(w, fmt, cache)
+    q = w.queries()
+    for b in range(w.batch):
+        one = gpu_decode(w, fmt, cache, q=q[b:b + 1], page_table=w.page_table[b:b + 1],
+                         seq_lens=w.seq_lens[b:b + 1])
+        assert np.array_equal(one[0], full[b])
+
+
+def test_page_permutation_invariance():
+    """Moving pages to other physical slots changes nothing, bit for bit."""
+    w = small(4, seq_lens=(700, 300))
+    cache = gpu_fill(w, 4)
+    out = gpu_decode(w, 4, cache)
+    perm = np.random.default_rng(3).permutation(w.num_pages)
+    from quantized_paged_kv_tq_b200 import tq as T
+    c2 = T.Cache(4, w.num_pages, w.num_kv_heads, w.page_size)
+    inv = torch.as_tensor(perm, device="cuda")
+    c2.k_pages[inv] = cache.k_pages
+    c2.v_pages[inv] = cache.v_pages
+    pt = np.where(w.page_table >= 0, perm[np.maximum(w.page_table, 0)], -1)
+    assert np.array_equal(gpu_decode(w, 4, c2, page_table=pt), out)
+
+
+def test_shared_prefix_equals_private_copies():
+    """Sequences reading one physical copy of a prefix give the same bits as
+    sequences holding private copies of the same prefix values."""
+    shared = W.custom(batch=3, seq_lens=(600, 900, 1100), q_len=4, num_q_heads=8,
+                      num_kv_heads=2, shared_prefix_seqs=3, shared_prefix_tokens=512,
+                      permute_pages=False, fmt=4, seed=9)
+    cache = gpu_fill(shared, 4)
+    out = gpu_decode(shared, 4, cache)
+    # private layout: copy the prefix pages for sequences 1 and 2
+    from quantized_paged_kv_tq_b200 import tq as T
+    P = shared.page_size
+    npre = 512 // P
+    extra = 2 * npre
+    c2 = T.Cache(4, shared.num_pages + extra, 2, P)
+    c2.k_pages[:shared.num_pages] = cache.k_pages
+    c2.v_pages[:shared.num_pages] = cache.v_pages
+    pt = shared.page_table.copy()
+    for i, b in enumerate((1, 2)):
+        new = shared.num_pages + i * npre + np.arange(npre)
+        c2.k_pages[torch.as_tensor(new, device="cuda")] = cache.k_pages[:npre]
+        c2.v_pages[torch.as_tensor(new, device="cuda")] = cache.v_pages[:npre]
+        pt[b, :npre] = new
+    assert np.array_equal(gpu_decode(shared, 4, c2, page_table=pt), out)
+    check_close(out, oracle_decode(shared, 4, np.arange(3)))
+
+
+def test_append_order_independence():
+    w = small(3, seq_lens=(500, 77))
+    a = gpu_fill(w, 3)
+    b = gpu_fill(w, 3, shuffle_seed=1)
+    c = gpu_fill(w, 3, chunk=7)
+    for x in (b, c):
+        assert torch.equal(a.k_pages, x.k_pages) and torch.equal(a.v_pages, x.v_pages)
+
+
+def test_causal_last_split_fully_masked_rows():
+    """seq_len 514 with q_len 4: the second split holds keys 512-513 only,
+    which rows t = 0, 1 must not see (their partial is empty)."""
+    w = small(4, q_len=4, seq_lens=(514, 516), batch=2)
+    cache = gpu_fill(w, 4)
+    check_close(gpu_decode(w, 4, cache), oracle_decode(w, 4, np.arange(2)))
+
+
+def test_repeated_calls_reuse_workspace():
+    """The merge counters return to zero: many calls on one workspace agree."""
+    w = small(4)
+    cache = gpu_fill(w, 4)
+    first = gpu_decode(w, 4, cache)
+    for _ in range(5):
+        assert np.array_equal(gpu_decode(w, 4, cache), first)
+
+
+# ------------------------------------------------------- device findings
+def test_device_checks_report_and_skip():
+    from quantized_paged_kv_tq_b200 import tq as T
+    w = small(4, seq_lens=(100, 40))
+    cache = gpu_fill(w, 4)
+    assert cache.read_error() == 0
+    # slot past the pool: skipped, reported
+    k = dev_bf16(np.zeros((1, 2, 128), np.uint16))
+    T.tq_quantize_append(k, k, dev(np.array([w.num_pages * 16 + 3], np.int64)), 4, cache)
+    code = cache.read_error()
+    assert code & 0xff == T.TQ_ERR_DEVICE_CHECK and code >> 8 == 1
+    # page-table entry out of range: reported
+    pt = w.page_table.copy()
+    pt[1, 0] = w.num_pages + 5
+    gpu_decode(w, 4, cache, page_table=pt)
+    code = cache.read_error()
+    assert code & 0xff == T.TQ_ERR_DEVICE_CHECK and code >> 8 == 2
+    # seq_len above max_seq_len: reported, sequence skipped
+    out = torch.zeros((2, 1, 8, 128), device="cuda")
+    sl = dev(np.array([100, 40], np.int32))
+    T.tq_paged_decode(dev_bf16(w.queries()), cache, dev(w.page_table), sl, 1, out,
+                      max_seq_len=50)
+    code = cache.read_error()
+    assert code & 0xff == T.TQ_ERR_DEVICE_CHECK and code >> 8 == 3
+    assert cache.read_error() == 0
+
+
+def test_empty_batch_and_zero_tokens():
+    from quantized_paged_kv_tq_b200 import tq as T
+    cache = T.Cache(4, 4, 2, 16)
+    e = torch.empty((0, 2, 128), dtype=torch.bfloat16, device="cuda")
+    T.tq_quantize_append(e, e, torch.empty(0, dtype=torch.int64, device="cuda"), 4, cache)
+    out = torch.empty((0, 1, 8, 128), device="cuda")
+    T.tq_paged_decode(torch.empty((0, 1, 8, 128), dtype=torch.bfloat16, device="cuda"), cache,
+                      torch.zeros((0, 4), dtype=torch.int32, device="cuda"),
+                      torch.zeros(0, dtype=torch.int32, device="cuda"), 1, out, max_seq_len=64)
+    torch.cuda.synchronize()
+    assert not cache.k_pages.any()
+
+
+def test_hbm_probes():
+    from quantized_paged_kv_tq_b200 import tq as T
+    src = torch.randint(0, 255, (1 << 24,), dtype=torch.uint8, device="cuda")
+    dst = torch.zeros_like(src)
+    T.tq_hbm_copy(src, dst)
+    sink = torch.zeros(1, dtype=torch.int32, device="cuda")
+    T.tq_hbm_read(src, sink)
+    torch.cuda.synchronize()
+    assert torch.equal(src, dst)
