@@ -608,8 +608,10 @@ k_decode(const DecodeArgs a)
                 const float p0 = sc[nt][e] == -CUDART_INF_F ? 0.f : exp2f(sc[nt][e] - m_run[nt][e]);
                 const float p1 = sc[nt][2 + e] == -CUDART_INF_F ? 0.f : exp2f(sc[nt][2 + e] - m_run[nt][e]);
                 l_run[nt][e] += p0 + p1;
-                pv[e] = p0 * vn0;
-                pv[2 + e] = p1 * vn1;
+                // a token masked for this row may carry a V scale above the
+                // running exponent: select, so 0 * (overflowed scale) is not NaN
+                pv[e] = p0 > 0.f ? p0 * vn0 : 0.f;
+                pv[2 + e] = p1 > 0.f ? p1 * vn1 : 0.f;
             }
             uint32_t top, bot;
             if constexpr (F::kTurbo) {
