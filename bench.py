@@ -315,6 +315,7 @@ def run_ours(args):
     read_gbs = nbytes / (min(read_ms) * 1e-3) / 1e9
     del a, bbuf
     torch.cuda.synchronize()
+    torch.cuda.empty_cache()
 
     # ---- warm-up
     for i in range(args.warmup):
