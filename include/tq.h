@@ -30,8 +30,10 @@
  *   within the page), then page_size fp32 scales.  BF16 block: page_size rows
  *   of d bf16 values.  A token's slot is page * page_size + offset.
  *
- * Ownership.  The library allocates nothing and keeps no state between calls.
- * Every buffer is caller-owned device memory unless stated otherwise.  Every
+ * Ownership.  The library allocates nothing and keeps no state between calls
+ * (the one exception is the fixed scratch array of tq_paged_decode_noalloc,
+ * described there).  Every buffer is caller-owned device memory unless
+ * stated otherwise.  Every
  * call is asynchronous on the given CUDA stream (a cudaStream_t passed as
  * void*, NULL = legacy default stream); calls on different streams are safe
  * when their buffers are disjoint.
@@ -194,6 +196,27 @@ tq_status tq_paged_decode_bf16(const void* q, const tq_cache* cache,
                                int32_t max_seq_len, float* out,
                                void* workspace, size_t workspace_bytes,
                                void* stream);
+
+/*
+ * tq_paged_decode_noalloc -- tq_paged_decode for callers that may not
+ * allocate device memory while they run (for example a runtime plugin whose
+ * enqueue hook works inside a fixed memory plan).  The pages have no
+ * counterpart; this is a convenience of this library.  Arguments as
+ * tq_paged_decode without the workspace: the split-KV scratch lives in one
+ * 64 MiB array inside libtq.so that every GPU loading the library holds
+ * until exit.  Shapes needing more than that return TQ_ERR_WORKSPACE before
+ * any launch.  The first call on a device looks the array up (so make it
+ * before any stream capture); every call clears the merge counters with a
+ * cudaMemsetAsync on `stream` and allocates nothing.  All calls share the
+ * array: calls that overlap in time on one GPU race and must be serialised
+ * by the caller.
+ */
+tq_status tq_paged_decode_noalloc(const void* q, const tq_cache* cache,
+                                  const int32_t* page_table,
+                                  int32_t max_pages_per_seq,
+                                  const int32_t* seq_lens, int32_t batch,
+                                  int32_t q_len, int32_t num_q_heads,
+                                  int32_t max_seq_len, float* out, void* stream);
 
 /*
  * tq_read_device_error -- wait (bounded, ~10 s) for the stream, then copy the

@@ -38,7 +38,7 @@ FORMATS = (TQ_TURBO2, TQ_TURBO3, TQ_TURBO4, TQ_TURBO8, TQ_BF16)
 SYMBOLS = ("tq_abi_version", "tq_status_string", "tq_page_block_bytes",
            "tq_quantize_append", "tq_append_bf16", "tq_decode_workspace_size",
            "tq_decode_workspace_init", "tq_paged_decode", "tq_paged_decode_bf16",
-           "tq_read_device_error", "tq_hbm_copy", "tq_hbm_read")
+           "tq_paged_decode_noalloc", "tq_read_device_error", "tq_hbm_copy", "tq_hbm_read")
 
 
 class tq_cache(ctypes.Structure):
@@ -69,6 +69,8 @@ _lib.tq_decode_workspace_init.argtypes = [_P, _S, _P]
 for _name in ("tq_paged_decode", "tq_paged_decode_bf16"):
     getattr(_lib, _name).restype = _I
     getattr(_lib, _name).argtypes = [_P, _CP, _P, _I, _P, _I, _I, _I, _I, _P, _P, _S, _P]
+_lib.tq_paged_decode_noalloc.restype = _I
+_lib.tq_paged_decode_noalloc.argtypes = [_P, _CP, _P, _I, _P, _I, _I, _I, _I, _P, _P]
 _lib.tq_read_device_error.restype = _I
 _lib.tq_read_device_error.argtypes = [_CP, ctypes.POINTER(ctypes.c_uint32), _I, _P]
 _lib.tq_hbm_copy.restype = _I
@@ -222,6 +224,21 @@ def tq_paged_decode_bf16(q, cache, page_table, seq_lens, q_len, out, max_seq_len
     """The same decode over a bf16 cache (uncompressed reference point)."""
     _decode(_lib.tq_paged_decode_bf16, "tq_paged_decode_bf16", q, cache, page_table, seq_lens,
             q_len, out, max_seq_len, workspace, stream)
+
+
+def tq_paged_decode_noalloc(q, cache, page_table, seq_lens, q_len, out, max_seq_len,
+                            stream=None) -> None:
+    """tq_paged_decode without a workspace argument, for callers that may not
+    allocate device memory while running: the scratch is a fixed 64 MiB array
+    inside libtq.so (shared by all calls, so overlapping calls on one GPU
+    must be serialised by the caller)."""
+    if q.shape[1] != q_len:
+        raise ValueError("q must be [batch][q_len][num_q_heads][head_dim]")
+    _check(_lib.tq_paged_decode_noalloc(
+        _dev(q, torch.bfloat16, "q"), ctypes.byref(_desc(cache)),
+        _dev(page_table, torch.int32, "page_table"), page_table.shape[1],
+        _dev(seq_lens, torch.int32, "seq_lens"), q.shape[0], q_len, q.shape[2], max_seq_len,
+        _dev(out, torch.float32, "out"), _stream(stream)), "tq_paged_decode_noalloc")
 
 
 def tq_read_device_error(cache, clear: bool = True, stream=None) -> int:
