@@ -26,9 +26,14 @@
  *
  * Cache layout in device memory (one pool for K, one for V, same shape):
  *   pool[num_pages][num_kv_heads][block], block = tq_page_block_bytes(...).
- *   turbo b-bit block: page_size rows of d*b/8 code bytes (row = token offset
- *   within the page), then page_size fp32 scales.  BF16 block: page_size rows
- *   of d bf16 values.  A token's slot is page * page_size + offset.
+ *   turbo b-bit K block: page_size token rows of d*b/8 code bytes (row t =
+ *   token t's packed vector), then page_size fp32 scales.
+ *   turbo b-bit V block: the same codes dim-major -- d rows of
+ *   page_size*b/8 bytes, row i holding every token's code i (token t at bits
+ *   [t*b, (t+1)*b) of the row, LSB-first) -- then page_size fp32 scales.
+ *   (K rows feed a decode thread per token, V rows a thread per dimension.)
+ *   BF16 block (K and V): page_size token rows of d bf16 values.
+ *   A token's slot is page * page_size + offset.
  *
  * Ownership.  The library allocates nothing and keeps no state between calls
  * (the one exception is the fixed scratch array of tq_paged_decode_noalloc,
@@ -173,9 +178,9 @@ tq_status tq_decode_workspace_init(void* workspace, size_t workspace_bytes,
  *                    when that size is 0), 16-byte aligned, initialised once
  *                    by tq_decode_workspace_init.  Calls that overlap in
  *                    time must use different workspaces.
- * Each sequence is split into fixed 512-token (page_size 16/32) or
- * 1024-token (page_size 64) parts whatever the batch holds, so a
- * sequence's output does not depend on the other sequences of the batch.
+ * Each sequence is split into fixed parts of 2048 tokens (1024 for 64-token
+ * pages) whatever the batch holds, so a sequence's output does not depend
+ * on the other sequences of the batch.
  */
 tq_status tq_paged_decode(const void* q, const tq_cache* cache,
                           const int32_t* page_table, int32_t max_pages_per_seq,

@@ -36,10 +36,13 @@
  *   GQA        query head h reads kv head h / (num_q_heads / num_kv_heads).
  *
  * Cache layout (an interface, described in include/tq.h, implemented here
- * independently): for a turbo format with b bits, each (page, kv head) block
- * holds page_size rows of d*b/8 code bytes followed by page_size fp32
- * scales; blocks are ordered [page][kv_head].  For BF16 each block holds
- * page_size rows of d bf16 values.  slot = page * page_size + offset.
+ * independently): blocks are ordered [page][kv_head].  For a turbo format
+ * with b bits and page size P, a K block holds P token rows of d*b/8 code
+ * bytes (row t = token t's packed vector as above) followed by P fp32
+ * scales.  A V block holds the same codes dim-major: d rows of P*b/8 bytes,
+ * row i packing the P tokens' codes of dimension i LSB-first (token t at
+ * bits [t*b, (t+1)*b) of the row), followed by the P fp32 scales.  For BF16
+ * each block holds P token rows of d bf16 values.  slot = page * P + offset.
  */
 #include <math.h>
 #include <stdint.h>
@@ -170,6 +173,28 @@ ORACLE_API void oracle_unpack_codes(const uint8_t* in, int d, int bits,
     }
 }
 
+/* Write / read an nbits-wide unsigned field at bit position `bit` of a
+ * little-endian byte string, one bit at a time. */
+static void put_bits(uint8_t* base, int64_t bit, int nbits, uint32_t value)
+{
+    for (int k = 0; k < nbits; ++k) {
+        int64_t b = bit + k;
+        uint8_t m = (uint8_t)(1u << (b % 8));
+        if ((value >> k) & 1u) base[b / 8] |= m;
+        else base[b / 8] &= (uint8_t)~m;
+    }
+}
+
+static uint32_t get_bits(const uint8_t* base, int64_t bit, int nbits)
+{
+    uint32_t v = 0;
+    for (int k = 0; k < nbits; ++k) {
+        int64_t b = bit + k;
+        v |= (uint32_t)((base[b / 8] >> (b % 8)) & 1u) << k;
+    }
+    return v;
+}
+
 /* Rotate, quantise and pack one bf16 head vector. */
 ORACLE_API void oracle_quantize_vector(const uint16_t* x_bf16, int d, int bits,
                                        uint8_t* packed, float* scale)
@@ -197,24 +222,36 @@ ORACLE_API int oracle_quantize_append(const uint16_t* k, const uint16_t* v,
     int64_t bb = oracle_block_bytes_impl(bits, d, page_size);
     if (bb < 0) return OR_BAD_ARG;
     const int cb = d * bits / 8;
-    for (int t = 0; t < num_tokens; ++t) {
+    float* y = (float*)malloc(sizeof(float) * (size_t)d);
+    int32_t* codes = (int32_t*)malloc(sizeof(int32_t) * (size_t)d);
+    int rc = OR_OK;
+    for (int t = 0; t < num_tokens && rc == OR_OK; ++t) {
         int64_t slot = slot_mapping[t];
         if (slot < 0) continue;
         int64_t page = slot / page_size;
         int64_t off = slot % page_size;
-        if (page >= num_pages) return OR_BAD_SLOT;
+        if (page >= num_pages) { rc = OR_BAD_SLOT; break; }
         for (int h = 0; h < num_kv_heads; ++h) {
             size_t blk = (size_t)((page * num_kv_heads + h) * bb);
             const uint16_t* kx = k + ((size_t)t * num_kv_heads + h) * d;
             const uint16_t* vx = v + ((size_t)t * num_kv_heads + h) * d;
             float ks, vs;
+            /* K: the token's packed vector is row `off` of the block */
             oracle_quantize_vector(kx, d, bits, k_pages + blk + off * cb, &ks);
-            oracle_quantize_vector(vx, d, bits, v_pages + blk + off * cb, &vs);
+            /* V: code i goes to row i (dim-major), field `off` */
+            oracle_rotate_f32(vx, d, y);
+            oracle_quantize_rotated(y, d, bits, codes, &vs);
+            const int L = (1 << (bits - 1)) - 1;
+            for (int i = 0; i < d; ++i)
+                put_bits(v_pages + blk, (int64_t)i * page_size * bits + (int64_t)off * bits,
+                         bits, (uint32_t)(codes[i] + L));
             memcpy(k_pages + blk + (size_t)page_size * cb + off * 4, &ks, 4);
             memcpy(v_pages + blk + (size_t)page_size * cb + off * 4, &vs, 4);
         }
     }
-    return OR_OK;
+    free(codes);
+    free(y);
+    return rc;
 }
 
 /* Store bf16 rows unchanged into a BF16 paged cache. */
@@ -239,17 +276,24 @@ ORACLE_API int oracle_append_bf16(const uint16_t* k, const uint16_t* v,
     return OR_OK;
 }
 
-/* Dequantised (still rotated) head vector of one cached token, fp64. */
+/* Dequantised (still rotated) head vector of one cached token, fp64.
+ * dim_major selects the V block layout (dimension rows of token fields). */
 static void dequant_token(const uint8_t* pages, int64_t bb, int page, int kvh,
                           int num_kv_heads, int off, int page_size, int d,
-                          int bits, int32_t* codes, double* out)
+                          int bits, int dim_major, int32_t* codes, double* out)
 {
     const int L = (1 << (bits - 1)) - 1;
     const int cb = d * bits / 8;
     const uint8_t* blk = pages + (size_t)(((int64_t)page * num_kv_heads + kvh) * bb);
     float s;
     memcpy(&s, blk + (size_t)page_size * cb + (size_t)off * 4, 4);
-    oracle_unpack_codes(blk + (size_t)off * cb, d, bits, codes);
+    if (dim_major) {
+        for (int i = 0; i < d; ++i)
+            codes[i] = (int32_t)get_bits(blk, (int64_t)i * page_size * bits +
+                                                  (int64_t)off * bits, bits) - L;
+    } else {
+        oracle_unpack_codes(blk + (size_t)off * cb, d, bits, codes);
+    }
     for (int i = 0; i < d; ++i)
         out[i] = (double)codes[i] * (double)s / (double)L;
 }
@@ -369,10 +413,10 @@ ORACLE_API int oracle_paged_decode(const uint16_t* q, int format, int d,
                     if (bits > 0) {
                         dequant_token((const uint8_t*)k_pages, bb, page, kvh,
                                       num_kv_heads, j % page_size, page_size, d,
-                                      bits, codes, kr);
+                                      bits, 0, codes, kr);
                         dequant_token((const uint8_t*)v_pages, bb, page, kvh,
                                       num_kv_heads, j % page_size, page_size, d,
-                                      bits, codes, vr);
+                                      bits, 1, codes, vr);
                     } else {
                         bf16_token((const uint16_t*)k_pages, page, kvh,
                                    num_kv_heads, j % page_size, page_size, d, kr);

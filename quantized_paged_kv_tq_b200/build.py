@@ -22,7 +22,7 @@ CSRC = os.path.join(PKG, "csrc")
 OUT = os.path.join(PKG, "libtq.so")
 OBJ = os.path.join(ROOT, "_build", "libtq")
 
-SOURCES = ["append.cu", "decode.cu", "decode_noalloc.cu", "api.cu", "hbm.cu"]
+SOURCES = ["append.cu", "decode.cu", "decode_tc.cu", "decode_noalloc.cu", "api.cu", "hbm.cu"]
 PER_FILE = {"append.cu": ["-fmad=false"]}
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",

@@ -17,9 +17,9 @@ cudaError_t launch_quantize_append(const void* k, const void* v, const int64_t* 
 cudaError_t launch_append_bf16(const void* k, const void* v, const int64_t* slots,
                                int num_tokens, const tq_cache& c, cudaStream_t stream);
 int decode_split_tokens(int page_size);
-int decode_row_groups(int G);
+int decode_row_groups(int format, int G);
 size_t decode_workspace_bytes(int batch, int num_kv_heads, int G, int max_seq_len,
-                              int page_size);
+                              int page_size, int format);
 cudaError_t launch_decode(const void* q, const tq_cache& c, int64_t block_bytes,
                           const int32_t* page_table, int max_pages, const int32_t* seq_lens,
                           int batch, int q_len, int num_q_heads, int max_seq_len, float* out,
@@ -102,14 +102,15 @@ tq_status check_decode(const void* q, const tq_cache* c, const int32_t* page_tab
     const int64_t G = (int64_t)q_len * (num_q_heads / c->num_kv_heads);
     if (G > kMaxRows) return TQ_ERR_UNSUPPORTED;
     if (batch > 65535) return TQ_ERR_UNSUPPORTED;
-    if ((int64_t)c->num_kv_heads * tq::decode_row_groups((int)G) > 65535) return TQ_ERR_UNSUPPORTED;
+    if ((int64_t)c->num_kv_heads * tq::decode_row_groups(c->format, (int)G) > 65535)
+        return TQ_ERR_UNSUPPORTED;
     if (batch == 0) return TQ_OK;
     if (!q || !page_table || !seq_lens || !out) return TQ_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(out) || (reinterpret_cast<uintptr_t>(page_table) & 3u) ||
         (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
         return TQ_ERR_INVALID_ARG;
     const size_t need = tq::decode_workspace_bytes(batch, c->num_kv_heads, (int)G, max_seq_len,
-                                                   c->page_size);
+                                                   c->page_size, c->format);
     if (need > 0) {
         if (!workspace || workspace_bytes < need) return TQ_ERR_WORKSPACE;
         if (!aligned16(workspace)) return TQ_ERR_INVALID_ARG;
@@ -185,7 +186,7 @@ TQ_API size_t tq_decode_workspace_size(int32_t batch, int32_t q_len, int32_t num
     const int64_t G = (int64_t)q_len * (num_q_heads / cache->num_kv_heads);
     if (G > kMaxRows) return 0;
     return tq::decode_workspace_bytes(batch, cache->num_kv_heads, (int)G, max_seq_len,
-                                      cache->page_size);
+                                      cache->page_size, cache->format);
 }
 
 TQ_API tq_status tq_decode_workspace_init(void* workspace, size_t workspace_bytes, void* stream)

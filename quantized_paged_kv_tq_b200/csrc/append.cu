@@ -98,6 +98,35 @@ __device__ __forceinline__ void store_codes(uint8_t* dst, const uint32_t u[4], i
     }
 }
 
+// Dim-major V rows: dimension i's row holds page_size fields of BITS bits,
+// token t at bits [t*BITS, (t+1)*BITS).  Tokens of one page may be appended
+// concurrently, so sub-byte fields are written with 32-bit atomic and/or
+// (each field is owned by one token; the other bits are left alone).
+template <int BITS>
+__device__ __forceinline__ void store_dim_major(uint8_t* blk, const uint32_t u[4], int lane,
+                                                int off, int page_size)
+{
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int i = 4 * lane + e;
+        const int64_t bit = (int64_t)i * page_size * BITS + (int64_t)off * BITS;
+        if constexpr (BITS == 8) {
+            blk[bit >> 3] = (uint8_t)u[e];
+        } else {
+            unsigned* w = reinterpret_cast<unsigned*>(blk) + (bit >> 5);
+            const int sh = (int)(bit & 31);
+            const unsigned field = (1u << BITS) - 1u;
+            atomicAnd(w, ~(field << sh));
+            atomicOr(w, u[e] << sh);
+            if (sh + BITS > 32) {            // a 3-bit field across two words
+                const int rest = sh + BITS - 32;
+                atomicAnd(w + 1, ~((1u << rest) - 1u));
+                atomicOr(w + 1, u[e] >> (BITS - rest));
+            }
+        }
+    }
+}
+
 template <int BITS>
 __global__ void __launch_bounds__(32 * kAppendWarps)
 k_quantize_append(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
@@ -155,7 +184,13 @@ k_quantize_append(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v
     }
 
     uint8_t* blk = (which ? vp : kp) + (page * num_kv_heads + head) * block_bytes;
-    store_codes<BITS>(blk + (int64_t)off * CB, u, lane);
+    if (!which) {
+        // K: the packed vector is token row `off`
+        store_codes<BITS>(blk + (int64_t)off * CB, u, lane);
+    } else {
+        // V: dim-major rows; code i is field `off` of row i
+        store_dim_major<BITS>(blk, u, lane, off, page_size);
+    }
     if (lane == 0)
         *reinterpret_cast<float*>(blk + (int64_t)page_size * CB + 4 * off) = s;
 }

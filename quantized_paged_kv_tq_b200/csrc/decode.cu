@@ -8,7 +8,7 @@
 // Work decomposition (split-KV):
 //   grid = (max splits, kv heads x row groups, batch), 4 warps per CTA.
 //   A CTA owns one (sequence, kv head, row group, split); a split is a fixed
-//   run of 512 tokens (1024 for 64-token pages), so a sequence's result
+//   run of 2048 tokens (1024 for 64-token pages), so a sequence's result
 //   never depends on the rest of the batch.  All G = q_len * GQA query rows
 //   of the kv head (up to 8 per row group) share every byte read.
 //   Each warp streams its own 16-token tiles (tile w, w+4, ...) through a
@@ -38,9 +38,29 @@ namespace tq {
 
 namespace {
 
+// Tuning constants (compile-time; the defaults are the measured choice).
+#ifndef TQ_SPLIT_TOKENS
+#define TQ_SPLIT_TOKENS 2048      // tokens per split-KV part (pages of 16/32), <= 2048
+#endif
+#ifndef TQ_SPLIT_TOKENS_P64
+#define TQ_SPLIT_TOKENS_P64 1024  // 64-token pages: >= 128 parts for a 131072-token context
+#endif
+#ifndef TQ_STAGE_BUDGET
+#define TQ_STAGE_BUDGET 6528      // target bytes of one warp's staging ring
+#endif
+#ifndef TQ_MAX_STAGES
+#define TQ_MAX_STAGES 3
+#endif
+static_assert(TQ_SPLIT_TOKENS % 64 == 0 && TQ_SPLIT_TOKENS <= 2048 &&
+                  TQ_SPLIT_TOKENS_P64 % 64 == 0 && TQ_SPLIT_TOKENS_P64 <= 2048,
+              "a warp holds the page ids of its tiles in one register per lane");
+
 constexpr int kWarps = 4;
 constexpr int kThreads = 32 * kWarps;
-constexpr int kMaxStages = 4;
+constexpr int kMaxStages = TQ_MAX_STAGES;
+// shared memory header: q rows [8][128] fp32, row factors, flags, mbarriers
+constexpr int kBarOff = 4224;
+constexpr int kRingOff = (kBarOff + 8 * 4 * kMaxStages + 127) / 128 * 128;
 constexpr int kRowsPerCta = 8;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazyThreshold = 8.f;       // log2 units
@@ -315,13 +335,19 @@ __device__ __forceinline__ void unpack_v(const uint8_t* codes, int g, int t, uin
 
 template <int BITS>
 __device__ __forceinline__ void issue_tile(uint8_t* dst, uint64_t* bar, const DecodeArgs& a,
-                                           int page, int kvh, int sub)
+                                           int page, int kvh, int sub, bool one_block)
 {
     using F = Fmt<BITS>;
     const int64_t blk = ((int64_t)page * a.num_kv_heads + kvh) * a.block_bytes;
     const uint8_t* kb = a.kp + blk;
     const uint8_t* vb = a.vp + blk;
     mbar_arrive_expect_tx(bar, F::kStageBytes);
+    if (one_block) {
+        // a 16-token page is exactly one tile: codes then scales, as staged
+        bulk_g2s(dst, kb, F::kVOff, bar);
+        bulk_g2s(dst + F::kVOff, vb, F::kVOff, bar);
+        return;
+    }
     bulk_g2s(dst, kb + sub * F::kTileCodes, F::kTileCodes, bar);
     bulk_g2s(dst + F::kVOff, vb + sub * F::kTileCodes, F::kTileCodes, bar);
     if constexpr (F::kTurbo) {
@@ -329,30 +355,6 @@ __device__ __forceinline__ void issue_tile(uint8_t* dst, uint64_t* bar, const De
         bulk_g2s(dst + F::kTileCodes, kb + so, 64, bar);
         bulk_g2s(dst + F::kVOff + F::kTileCodes, vb + so, 64, bar);
     }
-}
-
-__device__ __forceinline__ void fwht128_lane(float x[4], int lane)
-{
-    float a0 = x[0] + x[1], a1 = x[0] - x[1], a2 = x[2] + x[3], a3 = x[2] - x[3];
-    x[0] = a0 + a2;
-    x[2] = a0 - a2;
-    x[1] = a1 + a3;
-    x[3] = a1 - a3;
-#pragma unroll
-    for (int m = 1; m < 32; m <<= 1) {
-        const bool upper = (lane & m) != 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float p = __shfl_xor_sync(kFull, x[e], m);
-            x[e] = upper ? p - x[e] : x[e] + p;
-        }
-    }
-}
-
-__device__ __forceinline__ float pow2i(int e)  // 2^e for -126 <= e <= 127
-{
-    e = max(-126, min(127, e));
-    return __uint_as_float((uint32_t)(e + 127) << 23);
 }
 
 template <int BITS, int NT>
@@ -364,8 +366,8 @@ k_decode(const DecodeArgs a)
     float* sQ = reinterpret_cast<float*>(smem);                      // [8][128]
     float* sRowFac = sQ + kRowsPerCta * kHeadDim;                    // [8]
     int* sFlag = reinterpret_cast<int*>(sRowFac + 16);               // [4]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 4352 - 128); // [4][kMaxStages]
-    uint8_t* ring = smem + 4352;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);    // [4][kMaxStages]
+    uint8_t* ring = smem + kRingOff;
 
     const int split = blockIdx.x;
     const int b = blockIdx.z;
@@ -411,7 +413,9 @@ k_decode(const DecodeArgs a)
     for (int i = 0; i < first; ++i) {
         const int p = __shfl_sync(kFull, pid, i);
         const int sb = __shfl_sync(kFull, psub, i);
-        if (lane == 0) issue_tile<BITS>(myring + i * F::kStageBytes, &mybar[i], a, p, kvh, sb);
+        if (lane == 0)
+            issue_tile<BITS>(myring + i * F::kStageBytes, &mybar[i], a, p, kvh, sb,
+                             a.page_size == 16);
     }
 
     // ---- rotated, scaled query rows of this row group (while tiles load)
@@ -502,28 +506,38 @@ k_decode(const DecodeArgs a)
             l_run[nt][e] = 0.f;
         }
     }
-    int ev = 0;   // running biased fp32 exponent of the V scales (turbo)
+    // V scales: P' = p * s_v / L * 2^(127 - ev) with ev the largest biased
+    // fp32 exponent of the scales seen so far, so P' stays below 2^9 in f16
+    int ev = 0;
+    float vn = 1.f;                              // 2^(127 - ev)
+    float vlimit = __uint_as_float(1u << 23);    // scales >= this raise ev
     const float kinv = F::kTurbo ? 1.f / (float)F::L : 1.f;
+    const int ra = perm(g), rb = perm(g + 8);
+    // a tile is fully visible when its last token is within the causal limit
+    // of the first (most restricted) row of this row group
+    const int lim_min = seq_len - a.q_len + (rg * kRowsPerCta) / a.group;
+    const bool one_block = a.page_size == 16;
 
     int failed_at = -1;
-    for (int i = 0; i < my_tiles; ++i) {
-        const int slot = i % stages;
-        if (!mbar_wait_bounded(&mybar[slot], (uint32_t)((i / stages) & 1), kWaitSpins)) {
+    int slot = 0;
+    uint32_t phase = 0;
+    int tok0 = tok_begin + 16 * warp;
+    for (int i = 0; i < my_tiles; ++i, tok0 += 16 * kWarps) {
+        if (!mbar_wait_bounded(&mybar[slot], phase, kWaitSpins)) {
             if (lane == 0) report_error(a.err, TQ_ERR_TIMEOUT, kErrWaitTile);
             failed_at = i;
             break;
         }
         const uint8_t* st = myring + slot * F::kStageBytes;
-        const int tok0 = tok_begin + 16 * (warp + kWarps * i);
-        const int ra = perm(g), rb = perm(g + 8);
 
-        // ---------------- S = K q'
+        // ---------------- S = K q'  (two independent accumulation chains)
         float s[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int k = 0; k < 4; ++k) s[nt][k] = 0.f;
         {
+            float s2[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) s[nt][k] = s2[nt][k] = 0.f;
             uint32_t ka[8][2], kb[8][2];
             unpack_k<BITS>(st + ra * F::CB, t, ka);
             unpack_k<BITS>(st + rb * F::CB, t, kb);
@@ -532,13 +546,21 @@ k_decode(const DecodeArgs a)
                 const uint32_t afr[4] = {ka[c][0], kb[c][0], ka[c][1], kb[c][1]};
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    if constexpr (F::kTurbo) mma_f16(s[nt], afr, qf[nt][c][0], qf[nt][c][1]);
-                    else mma_bf16(s[nt], afr, qf[nt][c][0], qf[nt][c][1]);
+                    float* acc = c < 4 ? s[nt] : s2[nt];
+                    if constexpr (F::kTurbo) mma_f16(acc, afr, qf[nt][c][0], qf[nt][c][1]);
+                    else mma_bf16(acc, afr, qf[nt][c][0], qf[nt][c][1]);
                 }
             }
+            // hi + lo columns (lanes t and t ^ 2)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    s[nt][k] += s2[nt][k];
+                    s[nt][k] += __shfl_xor_sync(kFull, s[nt][k], 2);
+                }
         }
-        // hi + lo columns, then scale to log2 units
-        float ks0 = 1.f, ks1 = 1.f, vs0 = 1.f, vs1 = 1.f;
+        float ks0 = kinv, ks1 = kinv, vs0 = 1.f, vs1 = 1.f;
         if constexpr (F::kTurbo) {
             const float* kscale = reinterpret_cast<const float*>(st + F::kTileCodes);
             const float* vscale = reinterpret_cast<const float*>(st + F::kVOff + F::kTileCodes);
@@ -547,33 +569,43 @@ k_decode(const DecodeArgs a)
             vs0 = vscale[ra] * kinv;
             vs1 = vscale[rb] * kinv;
         }
+        const bool full = tok0 + 15 <= lim_min;     // warp-uniform
         const int ja = tok0 + ra, jb = tok0 + rb;
-        // slots past the sequence end were never written: keep their
-        // (arbitrary) scales out of every product
-        if (ja >= seq_len) { ks0 = 0.f; vs0 = 0.f; }
-        if (jb >= seq_len) { ks1 = 0.f; vs1 = 0.f; }
+        if (!full) {
+            // slots past the sequence end were never written: keep their
+            // (arbitrary) scales out of every product
+            if (ja >= seq_len) { ks0 = 0.f; vs0 = 0.f; }
+            if (jb >= seq_len) { ks1 = 0.f; vs1 = 0.f; }
+        }
+        // scores in log2 units; masked entries -inf (only in partial tiles)
         float sc[NT][4];
         bool need = false;
-        int vexp = 0;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                const float s0 = s[nt][e] + __shfl_xor_sync(kFull, s[nt][e], 2);
-                const float s1 = s[nt][2 + e] + __shfl_xor_sync(kFull, s[nt][2 + e], 2);
-                const bool v0 = ja <= lim[nt][e], v1 = jb <= lim[nt][e];
-                sc[nt][e] = v0 ? s0 * ks0 * rowfac[nt][e] : -CUDART_INF_F;
-                sc[nt][2 + e] = v1 ? s1 * ks1 * rowfac[nt][e] : -CUDART_INF_F;
-                need |= fmaxf(sc[nt][e], sc[nt][2 + e]) > m_run[nt][e] + kLazyThreshold;
-                if constexpr (F::kTurbo) {
-                    if (v0) vexp = max(vexp, (int)((__float_as_uint(vs0) >> 23) & 0xFF));
-                    if (v1) vexp = max(vexp, (int)((__float_as_uint(vs1) >> 23) & 0xFF));
+                float x0 = s[nt][e] * (ks0 * rowfac[nt][e]);
+                float x1 = s[nt][2 + e] * (ks1 * rowfac[nt][e]);
+                if (!full) {
+                    x0 = ja <= lim[nt][e] ? x0 : -CUDART_INF_F;
+                    x1 = jb <= lim[nt][e] ? x1 : -CUDART_INF_F;
                 }
+                sc[nt][e] = x0;
+                sc[nt][2 + e] = x1;
+                need |= fmaxf(x0, x1) > m_run[nt][e] + kLazyThreshold;
             }
-        int ev_new = ev;
-        if constexpr (F::kTurbo) ev_new = max(ev, (int)__reduce_max_sync(kFull, (unsigned)vexp));
-        if (__any_sync(kFull, need) || ev_new != ev) {
-            const float av = F::kTurbo ? pow2i(ev - ev_new) : 1.f;
+        if constexpr (F::kTurbo) need |= fmaxf(vs0, vs1) >= vlimit;
+        if (__any_sync(kFull, need)) {
+            float av = 1.f;
+            if constexpr (F::kTurbo) {
+                // non-negative floats order like their bit patterns
+                const unsigned vb = __reduce_max_sync(kFull, __float_as_uint(fmaxf(vs0, vs1)));
+                const int ev_new = max(ev, (int)(vb >> 23));
+                av = pow2i(ev - ev_new);
+                ev = ev_new;
+                vn = pow2i(127 - ev);
+                vlimit = ev >= 254 ? CUDART_INF_F : __uint_as_float((uint32_t)(ev + 1) << 23);
+            }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -583,7 +615,7 @@ k_decode(const DecodeArgs a)
                     v = fmaxf(v, __shfl_xor_sync(kFull, v, 8));
                     v = fmaxf(v, __shfl_xor_sync(kFull, v, 16));
                     const float mn = fmaxf(m_run[nt][e], v);
-                    const float alpha = mn == -CUDART_INF_F ? 1.f : exp2f(m_run[nt][e] - mn);
+                    const float alpha = mn == -CUDART_INF_F ? 1.f : fast_exp2(m_run[nt][e] - mn);
                     m_run[nt][e] = mn;
                     l_run[nt][e] *= alpha;
                     const float ao = alpha * av;
@@ -593,11 +625,9 @@ k_decode(const DecodeArgs a)
                         o[nt][mt][2 + e] *= ao;
                     }
                 }
-            ev = ev_new;
         }
-        // P' = p * s_v / L * 2^-(ev-127), split into hi (lanes t < 2) and
+        // P' = p * s_v / L * 2^(127 - ev), split into hi (lanes t < 2) and
         // lo (t >= 2) halves, transposed onto the PV B fragment
-        const float vn = F::kTurbo ? pow2i(127 - ev) : 1.f;
         const float vn0 = vs0 * vn, vn1 = vs1 * vn;
         uint32_t pb[NT][2];
 #pragma unroll
@@ -605,38 +635,25 @@ k_decode(const DecodeArgs a)
             float pv[4];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                const float p0 = sc[nt][e] == -CUDART_INF_F ? 0.f : exp2f(sc[nt][e] - m_run[nt][e]);
-                const float p1 = sc[nt][2 + e] == -CUDART_INF_F ? 0.f : exp2f(sc[nt][2 + e] - m_run[nt][e]);
+                float p0 = fast_exp2(sc[nt][e] - m_run[nt][e]);
+                float p1 = fast_exp2(sc[nt][2 + e] - m_run[nt][e]);
+                if (!full) {
+                    // -inf - -inf would be NaN: masked entries are exactly 0
+                    p0 = sc[nt][e] == -CUDART_INF_F ? 0.f : p0;
+                    p1 = sc[nt][2 + e] == -CUDART_INF_F ? 0.f : p1;
+                }
                 l_run[nt][e] += p0 + p1;
-                // a token masked for this row may carry a V scale above the
-                // running exponent: select, so 0 * (overflowed scale) is not NaN
-                pv[e] = p0 > 0.f ? p0 * vn0 : 0.f;
-                pv[2 + e] = p1 > 0.f ? p1 * vn1 : 0.f;
-            }
-            uint32_t top, bot;
-            if constexpr (F::kTurbo) {
-                if (t < 2) {
-                    top = pack_half2(pv[0], pv[1]);
-                    bot = pack_half2(pv[2], pv[3]);
-                } else {
-                    top = pack_half2(pv[0] - __half2float(__float2half_rn(pv[0])),
-                                     pv[1] - __half2float(__float2half_rn(pv[1])));
-                    bot = pack_half2(pv[2] - __half2float(__float2half_rn(pv[2])),
-                                     pv[3] - __half2float(__float2half_rn(pv[3])));
-                }
-            } else {
-                if (t < 2) {
-                    top = pack_bf162(pv[0], pv[1]);
-                    bot = pack_bf162(pv[2], pv[3]);
-                } else {
-                    top = pack_bf162(pv[0] - __bfloat162float(__float2bfloat16_rn(pv[0])),
-                                     pv[1] - __bfloat162float(__float2bfloat16_rn(pv[1])));
-                    bot = pack_bf162(pv[2] - __bfloat162float(__float2bfloat16_rn(pv[2])),
-                                     pv[3] - __bfloat162float(__float2bfloat16_rn(pv[3])));
+                pv[e] = p0 * vn0;
+                pv[2 + e] = p1 * vn1;
+                if (!full) {
+                    // a masked token may carry a scale above the running
+                    // exponent: 0 * (overflowed scale) must stay 0
+                    pv[e] = p0 > 0.f ? pv[e] : 0.f;
+                    pv[2 + e] = p1 > 0.f ? pv[2 + e] : 0.f;
                 }
             }
-            pb[nt][0] = movmatrix_trans(top);
-            pb[nt][1] = movmatrix_trans(bot);
+            pb[nt][0] = movmatrix_trans(split_hi_lo<F::kTurbo>(pv[0], pv[1], t < 2));
+            pb[nt][1] = movmatrix_trans(split_hi_lo<F::kTurbo>(pv[2], pv[3], t < 2));
         }
 
         // ---------------- O^T += V^T P'
@@ -657,7 +674,12 @@ k_decode(const DecodeArgs a)
             const int p = __shfl_sync(kFull, pid, i + stages);
             const int sb = __shfl_sync(kFull, psub, i + stages);
             if (lane == 0)
-                issue_tile<BITS>(myring + slot * F::kStageBytes, &mybar[slot], a, p, kvh, sb);
+                issue_tile<BITS>(myring + slot * F::kStageBytes, &mybar[slot], a, p, kvh, sb,
+                                 one_block);
+        }
+        if (++slot == stages) {
+            slot = 0;
+            phase ^= 1u;
         }
     }
 
@@ -811,7 +833,7 @@ k_decode(const DecodeArgs a)
 template <int BITS>
 int stages_for()
 {
-    const int s = 9216 / Fmt<BITS>::kStageBytes;
+    const int s = TQ_STAGE_BUDGET / Fmt<BITS>::kStageBytes;
     return s < 2 ? 2 : (s > kMaxStages ? kMaxStages : s);
 }
 
@@ -820,7 +842,7 @@ size_t smem_for(int stages)
 {
     const size_t ring = (size_t)kWarps * stages * Fmt<BITS>::kStageBytes;
     const size_t merge = (size_t)kWarps * kRowsPerCta * (kHeadDim + 2) * sizeof(float);
-    return 4352 + (ring > merge ? ring : merge);
+    return kRingOff + (ring > merge ? ring : merge);
 }
 
 template <int BITS, int NT>
@@ -844,20 +866,40 @@ cudaError_t launch_one(DecodeArgs a, dim3 grid, cudaStream_t stream)
 
 }  // namespace
 
-int decode_split_tokens(int page_size) { return page_size >= 64 ? 1024 : 512; }
+int decode_split_tokens(int page_size)
+{
+    return page_size >= 64 ? TQ_SPLIT_TOKENS_P64 : TQ_SPLIT_TOKENS;
+}
 
-int decode_row_groups(int G) { return (G + kRowsPerCta - 1) / kRowsPerCta; }
+
+int decode_tc_rows(int G);
+cudaError_t launch_decode_tc(const void* q, const tq_cache& c, int64_t block_bytes,
+                             const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                             int batch, int q_len, int num_q_heads, int max_seq_len, float* out,
+                             void* workspace, int split_tokens, cudaStream_t stream);
+
+// Query rows per CTA: the tensor-core kernel (turbo formats) takes 8 or 16,
+// the warp-MMA kernel (bf16) 8.
+int decode_rows_per_cta(int format, int G) { return format == 16 ? kRowsPerCta : decode_tc_rows(G); }
+
+int decode_row_groups(int format, int G)
+{
+    const int rows = decode_rows_per_cta(format, G);
+    return (G + rows - 1) / rows;
+}
 
 // Workspace: [counters (256-byte aligned)][m,l partials][O partials]
-size_t decode_workspace_bytes(int batch, int num_kv_heads, int G, int max_seq_len, int page_size)
+size_t decode_workspace_bytes(int batch, int num_kv_heads, int G, int max_seq_len, int page_size,
+                              int format)
 {
     const int st = decode_split_tokens(page_size);
     const int64_t max_splits = (max_seq_len + st - 1) / st;
     if (max_splits <= 1) return 0;
-    const int64_t units = (int64_t)batch * num_kv_heads * decode_row_groups(G);
+    const int rows = decode_rows_per_cta(format, G);
+    const int64_t units = (int64_t)batch * num_kv_heads * decode_row_groups(format, G);
     const int64_t cnt = ((units * 4 + 255) / 256) * 256;
-    const int64_t ml = ((units * max_splits * kRowsPerCta * 8 + 255) / 256) * 256;
-    const int64_t ob = units * max_splits * kRowsPerCta * kHeadDim * 4;
+    const int64_t ml = ((units * max_splits * rows * 8 + 255) / 256) * 256;
+    const int64_t ob = units * max_splits * rows * kHeadDim * 4;
     return (size_t)(cnt + ml + ob);
 }
 
@@ -866,6 +908,10 @@ cudaError_t launch_decode(const void* q, const tq_cache& c, int64_t block_bytes,
                           int batch, int q_len, int num_q_heads, int max_seq_len, float* out,
                           void* workspace, cudaStream_t stream)
 {
+    if (c.format != 16)
+        return launch_decode_tc(q, c, block_bytes, page_table, max_pages, seq_lens, batch, q_len,
+                                num_q_heads, max_seq_len, out, workspace,
+                                decode_split_tokens(c.page_size), stream);
     DecodeArgs a{};
     a.q = static_cast<const uint16_t*>(q);
     a.kp = static_cast<const uint8_t*>(c.k_pages);
@@ -882,7 +928,7 @@ cudaError_t launch_decode(const void* q, const tq_cache& c, int64_t block_bytes,
     a.group = num_q_heads / c.num_kv_heads;
     a.q_len = q_len;
     a.G = q_len * a.group;
-    a.R = decode_row_groups(a.G);
+    a.R = decode_row_groups(16, a.G);
     a.page_size = c.page_size;
     a.split_tokens = decode_split_tokens(c.page_size);
     a.max_splits = (max_seq_len + a.split_tokens - 1) / a.split_tokens;

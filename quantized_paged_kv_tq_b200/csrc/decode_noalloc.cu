@@ -25,8 +25,8 @@
 
 namespace tq {
 size_t decode_workspace_bytes(int batch, int num_kv_heads, int G, int max_seq_len,
-                              int page_size);
-int decode_row_groups(int G);
+                              int page_size, int format);
+int decode_row_groups(int format, int G);
 cudaError_t launch_decode(const void* q, const tq_cache& c, int64_t block_bytes,
                           const int32_t* page_table, int max_pages, const int32_t* seq_lens,
                           int batch, int q_len, int num_q_heads, int max_seq_len, float* out,
@@ -96,7 +96,7 @@ TQ_API tq_status tq_paged_decode_noalloc(const void* q, const tq_cache* cache,
         return TQ_ERR_INVALID_ARG;
     const int64_t G = (int64_t)q_len * (num_q_heads / cache->num_kv_heads);
     if (G > 64 || batch > 65535) return TQ_ERR_UNSUPPORTED;
-    if ((int64_t)cache->num_kv_heads * tq::decode_row_groups((int)G) > 65535)
+    if ((int64_t)cache->num_kv_heads * tq::decode_row_groups(f, (int)G) > 65535)
         return TQ_ERR_UNSUPPORTED;
     if (batch == 0) return TQ_OK;
     if (!q || !page_table || !seq_lens || !out || !aligned16(q) || !aligned16(out) ||
@@ -105,7 +105,7 @@ TQ_API tq_status tq_paged_decode_noalloc(const void* q, const tq_cache* cache,
         return TQ_ERR_INVALID_ARG;
 
     const size_t need = tq::decode_workspace_bytes(batch, cache->num_kv_heads, (int)G,
-                                                   max_seq_len, cache->page_size);
+                                                   max_seq_len, cache->page_size, f);
     if (need > kStaticScratchBytes) return TQ_ERR_WORKSPACE;   // beyond the fixed maximum
 
     void* scratch = nullptr;
@@ -115,7 +115,8 @@ TQ_API tq_status tq_paged_decode_noalloc(const void* q, const tq_cache* cache,
         // The array keeps whatever the previous call left.  Only the merge
         // counters at its start must begin at zero; the partials are always
         // written before they are read.
-        const size_t units = (size_t)batch * cache->num_kv_heads * tq::decode_row_groups((int)G);
+        const size_t units =
+            (size_t)batch * cache->num_kv_heads * tq::decode_row_groups(f, (int)G);
         if (cudaMemsetAsync(scratch, 0, units * sizeof(uint32_t), s) != cudaSuccess)
             return TQ_ERR_CUDA;
     }

@@ -1,0 +1,752 @@
+// Paged decode / speculative-verify attention over a TurboQuant cache on the
+// 5th-generation tensor cores (tcgen05, tensor memory).
+//
+// "xInfer: Pure-Rust LLM Inference Without a Python Runtime", section
+// "TurboQuant is a memory trade": reading a low-bit KV cache dequantises on
+// every attention step.  "infero", section "Continuous batching": a running
+// batch shares the GPU over a paged KV cache.
+//
+// One CTA (128 threads) owns one (sequence, kv head, row group, split) with
+// splits of 2048 tokens (1024 for 64-token pages) fixed by the sequence
+// length alone.  The split is walked in tiles of 128 tokens; the K and V page
+// blocks of a tile arrive by 1-D bulk async copies into a 2-stage ring.
+// Per tile:
+//   1. thread t unpacks token t's K codes into exact f16 integers and stores
+//      them into tensor memory (lane t): the A operand of S = K q'.
+//   2. one thread issues S[128 tok][N] = A x Q' (Q' in shared memory: the
+//      rotated query, split into f16 hi and lo columns, N = 2 x rows).
+//   3. thread t reads its token's scores from tensor memory (hi + lo), scales
+//      them by s_k / L, and runs the online softmax (a lazy max: rescale only
+//      when a tile beats the running max by 2^8; one CTA-wide vote per tile).
+//      P' = p * s_v / L is written, split hi/lo in f16, to shared memory as
+//      the B operand of the PV product.
+//   4. thread d unpacks dimension d's V codes of the tile (the V block is
+//      dim-major) into tensor memory (lane d): A operand of O^T += V^T P'.
+//      The accumulator O^T lives in tensor memory for the whole split.
+// The epilogue merges the split (last CTA of a sequence/kv head wins an
+// atomic ticket and merges all splits), rotates back (H o / sqrt(d)) and
+// writes fp32 output.
+#include <cstdint>
+#include <math_constants.h>
+
+#include "tq_device.cuh"
+
+namespace tq {
+
+namespace {
+
+constexpr int kTcThreads = 128;
+constexpr int kTile = 128;               // tokens per tile (= tensor-memory lanes)
+constexpr int kStages = 2;
+constexpr uint32_t kTmemCols = 128;      // A: 64 columns, S: N, O: N (N <= 32)
+constexpr float kLog2eTc = 1.4426950408889634f;
+constexpr float kLazyTc = 8.f;
+constexpr uint32_t kSpinsTc = 1u << 24;
+constexpr uint32_t kMagicTc = 0x64006400u;
+
+struct TcArgs {
+    const uint16_t* q;
+    const uint8_t* kp;
+    const uint8_t* vp;
+    const int32_t* page_table;
+    const int32_t* seq_lens;
+    float* out;
+    float* ws_o;
+    float2* ws_ml;
+    uint32_t* ws_cnt;
+    uint32_t* err;
+    int64_t block_bytes;
+    int max_pages;
+    int num_pages;
+    int num_kv_heads;
+    int num_q_heads;
+    int group;
+    int q_len;
+    int G;
+    int R;             // row groups
+    int page_size;
+    int split_tokens;
+    int max_splits;
+    int max_seq_len;
+};
+
+template <int BITS>
+struct TcFmt {
+    static constexpr int CB = 16 * BITS;              // K row bytes (128 codes)
+    static constexpr int L = (1 << (BITS - 1)) - 1;
+    // codes come out of the unpacker in pairs (j, j + GB/2) of groups of GB
+    static constexpr int GB = BITS == 2 ? 16 : (BITS == 8 ? 4 : 8);
+    static constexpr int kStage = 2 * kTile * (CB + 4);   // K and V blocks of one tile
+};
+
+// Index (dimension for K, token for V) held at K position k of an A operand,
+// i.e. the order the unpacker emits: pair c holds (perm(2c), perm(2c + 1)).
+template <int GB>
+__device__ __forceinline__ int perm_k(int k)
+{
+    return (k / GB) * GB + ((k % GB) >> 1) + (GB / 2) * (k & 1);
+}
+template <int GB>
+__device__ __forceinline__ int perm_inv(int i)
+{
+    const int m = i % GB;
+    return (i / GB) * GB + (m < GB / 2 ? 2 * m : 2 * (m - GB / 2) + 1);
+}
+
+// f16x2 of (code a, code b) from magic-number halves: (1024 + 2^s u) * 2^-s - (1024 2^-s + L)
+__device__ __forceinline__ uint32_t mk(uint32_t bits_with_magic, uint32_t mul, uint32_t add)
+{
+    return hfma2_u32(bits_with_magic, mul, add);
+}
+
+// ---------------------------------------------------------------- unpack
+// Emit the pairs of one 32-bit word of 4-bit codes (8 codes): (0,4) (1,5) (2,6) (3,7).
+__device__ __forceinline__ void pairs4(uint32_t w, uint32_t* o)
+{
+    const uint32_t w8 = w >> 8;
+    o[0] = mk(and_or(w, 0x000F000Fu, kMagicTc), 0x3C003C00u, 0xE407E407u);
+    o[1] = mk(and_or(w, 0x00F000F0u, kMagicTc), 0x2C002C00u, 0xD470D470u);
+    o[2] = mk(and_or(w8, 0x000F000Fu, kMagicTc), 0x3C003C00u, 0xE407E407u);
+    o[3] = mk(and_or(w8, 0x00F000F0u, kMagicTc), 0x2C002C00u, 0xD470D470u);
+}
+// 8-bit codes (4 per word): (0,2) (1,3)
+__device__ __forceinline__ void pairs8(uint32_t w, uint32_t* o)
+{
+    o[0] = mk(prmt(w, 0x64646464u, 0x4240u), 0x3C003C00u, 0xE47FE47Fu);
+    o[1] = mk(prmt(w, 0x64646464u, 0x4341u), 0x3C003C00u, 0xE47FE47Fu);
+}
+// 2-bit codes (16 per word): (j, j+8), j = 0..7
+__device__ __forceinline__ void pairs2(uint32_t w, uint32_t* o)
+{
+    constexpr uint32_t mul[4] = {0x3C003C00u, 0x34003400u, 0x2C002C00u, 0x24002400u};
+    constexpr uint32_t add[4] = {0xE401E401u, 0xDC04DC04u, 0xD410D410u, 0xCC40CC40u};
+    const uint32_t w8 = w >> 8;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int jj = j & 3;
+        o[j] = mk(and_or(j < 4 ? w : w8, 0x00030003u << (2 * jj), kMagicTc), mul[jj], add[jj]);
+    }
+}
+// 3-bit codes: one 24-bit group of 8 codes (bits 0..23 of g): (k, k+4), k = 0..3
+__device__ __forceinline__ void pairs3(uint32_t g, uint32_t* o)
+{
+    constexpr uint32_t mul[3] = {0x3C003C00u, 0x30003000u, 0x24002400u};
+    constexpr uint32_t add[3] = {0xE403E403u, 0xD818D818u, 0xCCC0CCC0u};
+    const uint32_t sel = bitsel(g, g << 4, 0x0000FFFFu);
+    const uint32_t sel3 = bitsel(g >> 3, g << 1, 0x0000FFFFu);
+    o[0] = mk(and_or(sel, 0x00070007u, kMagicTc), mul[0], add[0]);
+    o[1] = mk(and_or(sel, 0x00380038u, kMagicTc), mul[1], add[1]);
+    o[2] = mk(and_or(sel, 0x01C001C0u, kMagicTc), mul[2], add[2]);
+    o[3] = mk(and_or(sel3, 0x01C001C0u, kMagicTc), mul[2], add[2]);
+}
+
+// K row of one token (128 codes) -> tensor memory columns [col, col + 64).
+template <int BITS>
+__device__ __forceinline__ void k_row_to_tmem(const uint8_t* row, uint32_t taddr)
+{
+    uint32_t o[16];
+    if constexpr (BITS == 4) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint4 w = *reinterpret_cast<const uint4*>(row + 16 * q);
+            pairs4(w.x, o);
+            pairs4(w.y, o + 4);
+            pairs4(w.z, o + 8);
+            pairs4(w.w, o + 12);
+            tmem_st16(taddr + 16 * q, o);
+        }
+    } else if constexpr (BITS == 8) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint4 a = *reinterpret_cast<const uint4*>(row + 32 * q);
+            const uint4 b = *reinterpret_cast<const uint4*>(row + 32 * q + 16);
+            pairs8(a.x, o); pairs8(a.y, o + 2); pairs8(a.z, o + 4); pairs8(a.w, o + 6);
+            pairs8(b.x, o + 8); pairs8(b.y, o + 10); pairs8(b.z, o + 12); pairs8(b.w, o + 14);
+            tmem_st16(taddr + 16 * q, o);
+        }
+    } else if constexpr (BITS == 2) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const uint4 w = *reinterpret_cast<const uint4*>(row + 16 * q);
+            pairs2(w.x, o);
+            pairs2(w.y, o + 8);
+            tmem_st16(taddr + 32 * q, o);
+            pairs2(w.z, o);
+            pairs2(w.w, o + 8);
+            tmem_st16(taddr + 32 * q + 16, o);
+        }
+    } else {  // 3 bits: 48-byte row, 12 words, 16 groups of 8 codes
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            // 12 bytes = 3 words = 4 groups
+            const uint32_t* p = reinterpret_cast<const uint32_t*>(row + 12 * q);
+            const uint32_t W0 = p[0], W1 = p[1], W2 = p[2];
+            pairs3(W0, o);
+            pairs3(prmt(W0, W1, 0x6543u), o + 4);
+            pairs3(prmt(W1, W2, 0x5432u), o + 8);
+            pairs3(W2 >> 8, o + 12);
+            tmem_st16(taddr + 16 * q, o);
+        }
+    }
+}
+
+// V codes of dimension `dim` for the 128 tokens of a tile -> tensor memory
+// columns [0, 64) of this thread's lane.  vblk0: first V block of the tile in
+// the stage; pages of P tokens follow each other every block_bytes.
+template <int BITS>
+__device__ __forceinline__ void v_col_to_tmem(const uint8_t* vblk0, int64_t bb, int P, int dim,
+                                              uint32_t taddr)
+{
+    uint32_t o[16];
+    // tokens are emitted 16 pairs (32 tokens) per store
+    const int row_bytes = P * BITS / 8;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int t0 = 32 * q;                   // first tile token of this chunk
+        const int pg = t0 / P;                   // page holding it
+        const int in = t0 % P;                   // its offset in the page
+        const uint8_t* row = vblk0 + pg * bb + (int64_t)dim * row_bytes;
+        if constexpr (BITS == 4) {
+            // 32 tokens = 16 bytes of one row (P >= 32) or two 8-byte rows (P = 16)
+            uint32_t w[4];
+            if (P >= 32) {
+                const uint4 x = *reinterpret_cast<const uint4*>(row + in / 2);
+                w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
+            } else {
+                const uint2 x = *reinterpret_cast<const uint2*>(row);
+                const uint2 y = *reinterpret_cast<const uint2*>(row + bb);
+                w[0] = x.x; w[1] = x.y; w[2] = y.x; w[3] = y.y;
+            }
+            pairs4(w[0], o); pairs4(w[1], o + 4); pairs4(w[2], o + 8); pairs4(w[3], o + 12);
+        } else if constexpr (BITS == 8) {
+            // 32 tokens = 32 bytes (P >= 32) or two 16-byte rows (P = 16)
+            uint4 x, y;
+            if (P >= 32) {
+                x = *reinterpret_cast<const uint4*>(row + in);
+                y = *reinterpret_cast<const uint4*>(row + in + 16);
+            } else {
+                x = *reinterpret_cast<const uint4*>(row);
+                y = *reinterpret_cast<const uint4*>(row + bb);
+            }
+            pairs8(x.x, o); pairs8(x.y, o + 2); pairs8(x.z, o + 4); pairs8(x.w, o + 6);
+            pairs8(y.x, o + 8); pairs8(y.y, o + 10); pairs8(y.z, o + 12); pairs8(y.w, o + 14);
+        } else if constexpr (BITS == 2) {
+            // 32 tokens = 8 bytes (P >= 32) or two 4-byte rows (P = 16)
+            uint32_t a, c;
+            if (P >= 32) {
+                const uint2 x = *reinterpret_cast<const uint2*>(row + in / 4);
+                a = x.x; c = x.y;
+            } else {
+                a = *reinterpret_cast<const uint32_t*>(row);
+                c = *reinterpret_cast<const uint32_t*>(row + bb);
+            }
+            pairs2(a, o);
+            pairs2(c, o + 8);
+        } else {
+            // 3 bits: 16 tokens are 6 bytes at a 2-byte boundary of the block;
+            // read the two aligned words around them and shift
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                // 16 tokens from a longer page, or the whole next 16-token page
+                const int tk = (P >= 32) ? in + 16 * h : 0;    // first token in its page
+                const int hp = (P >= 32) ? pg : pg + h;        // page of these 16
+                const int off = dim * row_bytes + 3 * tk / 8;  // byte offset in block
+                const uint32_t* wp =
+                    reinterpret_cast<const uint32_t*>(vblk0 + hp * bb + (off & ~3));
+                const uint64_t v64 = (((uint64_t)wp[1] << 32) | wp[0]) >> ((off & 3) * 8);
+                pairs3((uint32_t)v64 & 0xFFFFFFu, o + 8 * h);
+                pairs3((uint32_t)(v64 >> 24) & 0xFFFFFFu, o + 8 * h + 4);
+            }
+        }
+        tmem_st16(taddr + 16 * q, o);
+    }
+}
+
+// Bulk copies of one tile's K and V page blocks into a stage (warp 0).
+__device__ __forceinline__ void issue_tile_tc(uint8_t* stage, uint64_t* bar, const TcArgs& a,
+                                              int b, int kvh, int tok0, int ntok, int lane)
+{
+    const int P = a.page_size;
+    const int npp = kTile / P;                          // page slots per stage
+    const int npg = (ntok + P - 1) / P;                 // pages holding tokens
+    if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(2 * npg * a.block_bytes));
+    __syncwarp();
+    if (lane < npg) {
+        int pid = __ldg(a.page_table + (int64_t)b * a.max_pages + tok0 / P + lane);
+        if (pid < 0 || pid >= a.num_pages) {
+            report_error(a.err, TQ_ERR_DEVICE_CHECK, kErrPageRange);
+            pid = 0;
+        }
+        const int64_t off = ((int64_t)pid * a.num_kv_heads + kvh) * a.block_bytes;
+        bulk_g2s(stage + lane * a.block_bytes, a.kp + off, (uint32_t)a.block_bytes, bar);
+        bulk_g2s(stage + (npp + lane) * a.block_bytes, a.vp + off, (uint32_t)a.block_bytes, bar);
+    }
+}
+
+template <int BITS, int NCOL>
+__global__ void __launch_bounds__(kTcThreads, 4)
+k_decode_tc(const TcArgs a)
+{
+    using F = TcFmt<BITS>;
+    constexpr int RG = NCOL / 2;              // query rows per CTA
+    constexpr uint32_t kColS = 64, kColO = 64 + NCOL;
+    // instruction descriptors: f32 accumulate, f16 operands, M = 128, N = NCOL;
+    // B K-major (Q') for S, B MN-major (P') for O
+    constexpr uint32_t kIdescS = (1u << 4) | ((uint32_t)(NCOL >> 3) << 17) | (8u << 24);
+    constexpr uint32_t kIdescO = kIdescS | (1u << 16);
+    constexpr uint32_t kCmRow = (NCOL / 8) * 128;   // bytes per 8-deep K group
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);              // [kStages]
+    uint64_t* bar_s = full + kStages;
+    uint64_t* bar_o = bar_s + 1;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + 64);
+    int* s_flag = reinterpret_cast<int*>(smem + 68);                 // [0] abort, [1] ticket
+    float* s_red = reinterpret_cast<float*>(smem + 128);             // [4][16] row maxima
+    unsigned* s_redv = reinterpret_cast<unsigned*>(smem + 384);      // [4]
+    float* s_rowfac = reinterpret_cast<float*>(smem + 400);          // [16]
+    float* s_l = reinterpret_cast<float*>(smem + 464);               // [4][16]
+    uint8_t* s_qb = smem + 1024;                                     // Q' operand
+    uint8_t* s_pb = s_qb + 256 * NCOL;                               // P' operand / q staging
+    uint8_t* ring = s_pb + 256 * NCOL;
+
+    const int split = blockIdx.x;
+    const int b = blockIdx.z;
+    const int kvh = blockIdx.y / a.R;
+    const int rg = blockIdx.y - kvh * a.R;
+    const int seq_len = a.seq_lens[b];
+    if (seq_len < a.q_len || seq_len > a.max_seq_len) {
+        if (split == 0 && blockIdx.y == 0 && threadIdx.x == 0)
+            report_error(a.err, TQ_ERR_DEVICE_CHECK, kErrSeqLen);
+        return;
+    }
+    const int nsplit = (seq_len + a.split_tokens - 1) / a.split_tokens;
+    if (split >= nsplit) return;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tok_begin = split * a.split_tokens;
+    const int tok_end = min(seq_len, tok_begin + a.split_tokens);
+    const int ntiles = (tok_end - tok_begin + kTile - 1) / kTile;
+    const int P = a.page_size;
+    const int npp = kTile / P;
+
+    // ---- set-up: barriers, tensor memory, first copies
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+        mbar_init(bar_s, 1);
+        mbar_init(bar_o, 1);
+        s_flag[0] = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(s_tmem, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    const uint32_t t_lane = tmem + ((uint32_t)(32 * warp) << 16);   // this thread's lane
+
+    if (warp == 0) {
+        for (int s = 0; s < kStages && s < ntiles; ++s) {
+            const int t0 = tok_begin + s * kTile;
+            issue_tile_tc(ring + s * F::kStage, &full[s], a, b, kvh, t0, min(kTile, tok_end - t0),
+                          lane);
+        }
+    }
+
+    // ---- query rows of this row group: rotate, scale to log2 units,
+    // power-of-two prescale (hi and lo parts stay normal f16)
+    float* s_qf = reinterpret_cast<float*>(s_pb);                    // [RG][128]
+    for (int rr = warp; rr < RG; rr += 4) {
+        const int r = rg * RG + rr;
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        if (r < a.G) {
+            const int tq = r / a.group;
+            const int h = kvh * a.group + (r - tq * a.group);
+            const uint2 raw = __ldg(reinterpret_cast<const uint2*>(
+                a.q + (((int64_t)b * a.q_len + tq) * a.num_q_heads + h) * kHeadDim) + lane);
+            x[0] = bf16_bits_to_float(raw.x & 0xffffu);
+            x[1] = bf16_bits_to_float(raw.x >> 16);
+            x[2] = bf16_bits_to_float(raw.y & 0xffffu);
+            x[3] = bf16_bits_to_float(raw.y >> 16);
+        }
+        fwht128_lane(x, lane);
+        float amax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            x[e] *= kLog2eTc / kHeadDim;       // (H q / sqrt d) . y / sqrt d = (H q) . y / d
+            amax = fmaxf(amax, fabsf(x[e]));
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, m));
+        const int ex = amax > 0.f ? max(-100, min(100, ilogbf(amax))) : 0;
+        const float pre = pow2i(12 - ex);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s_qf[rr * kHeadDim + 4 * lane + e] = x[e] * pre;
+        if (lane == 0) s_rowfac[rr] = pow2i(ex - 12);
+    }
+    __syncthreads();
+    {
+        // Q' operand, K-major: K position k = tid holds dimension perm(k);
+        // column n < RG is row n's hi part, n >= RG its lo part
+        const int k = tid;
+        const int dim = perm_k<F::GB>(k);
+        __half* qb = reinterpret_cast<__half*>(s_qb);
+#pragma unroll
+        for (int n = 0; n < NCOL; ++n) {
+            const float v = s_qf[(n % RG) * kHeadDim + dim];
+            const float hi = __half2float(__float2half_rn(v));
+            const __half h = __float2half_rn(n < RG ? v : v - hi);
+            const int cm = (k >> 3) * (NCOL / 8) + (n >> 3);
+            qb[(cm * 128 + (n & 7) * 16 + (k & 7) * 2) / 2] = h;
+        }
+    }
+    float rowfac[RG];
+    int lim[RG];
+#pragma unroll
+    for (int r = 0; r < RG; ++r) {
+        rowfac[r] = s_rowfac[r];
+        const int R = rg * RG + r;
+        lim[r] = R < a.G ? seq_len - a.q_len + R / a.group : -1;
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+
+    float m_run[RG], l_run[RG];
+#pragma unroll
+    for (int r = 0; r < RG; ++r) {
+        m_run[r] = -CUDART_INF_F;
+        l_run[r] = 0.f;
+    }
+    int ev = 0;                                   // running V-scale exponent (biased)
+    float vn = 1.f;                               // 2^(127 - ev)
+    float vlimit = __uint_as_float(1u << 23);     // scales >= this raise ev
+    const float kinv = 1.f / (float)F::L;
+    const int lim_min = seq_len - a.q_len + (rg * RG) / a.group;
+    const int kpos = perm_inv<F::GB>(tid);        // this token's K position in PV
+    bool aborted = false;
+
+    for (int tt = 0; tt < ntiles; ++tt) {
+        const int stage = tt % kStages;
+        uint8_t* st = ring + stage * F::kStage;
+        const int tok0 = tok_begin + tt * kTile;
+        bool ok = mbar_wait_bounded(&full[stage], (uint32_t)((tt / kStages) & 1), kSpinsTc);
+        if (tt > 0) ok = ok && mbar_wait_bounded(bar_o, (uint32_t)((tt - 1) & 1), kSpinsTc);
+        tc_fence_after();
+        if (!ok) atomicOr(&s_flag[0], 1);
+
+        // 1. K row of token tid -> A operand
+        const int pg = tid / P, row = tid % P;
+        const uint8_t* kblk = st + pg * a.block_bytes;
+        const uint8_t* vblk = st + (npp + pg) * a.block_bytes;
+        k_row_to_tmem<BITS>(kblk + row * F::CB, t_lane);
+        float ks = reinterpret_cast<const float*>(kblk + P * F::CB)[row] * kinv;
+        float vs = reinterpret_cast<const float*>(vblk + P * F::CB)[row] * kinv;
+        const int tok = tok0 + tid;
+        if (tok >= tok_end) { ks = 0.f; vs = 0.f; }       // slot never written
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+        if (s_flag[0]) { aborted = true; break; }
+
+        // 2. S = K Q'
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                umma_f16_ts(tmem + kColS, tmem + 8 * j,
+                            smem_desc(s_qb + 2 * j * kCmRow, kCmRow, 128), kIdescS, j > 0);
+            umma_commit(bar_s);
+        }
+        ok = mbar_wait_bounded(bar_s, (uint32_t)(tt & 1), kSpinsTc);
+        tc_fence_after();
+        if (!ok) atomicOr(&s_flag[0], 1);
+
+        // 3. scores of token tid; V column of dimension tid -> A operand
+        uint32_t sraw[NCOL];
+#pragma unroll
+        for (int c = 0; c < NCOL; c += 16) tmem_ld16(t_lane + kColS + c, sraw + c);
+        v_col_to_tmem<BITS>(st + npp * a.block_bytes, a.block_bytes, P, tid, t_lane);
+        tmem_wait_ld();
+        const bool full_tile = tok0 + kTile - 1 <= lim_min;
+        float sc[RG];
+        bool need = false;
+#pragma unroll
+        for (int r = 0; r < RG; ++r) {
+            float x = (__uint_as_float(sraw[r]) + __uint_as_float(sraw[RG + r])) * (ks * rowfac[r]);
+            if (!full_tile) x = tok <= lim[r] ? x : -CUDART_INF_F;
+            sc[r] = x;
+            need |= x > m_run[r] + kLazyTc;
+        }
+        need |= vs >= vlimit;
+        const int any = __syncthreads_or(need);          // also: the stage is consumed
+        if (s_flag[0]) { aborted = true; break; }
+        if (warp == 0 && tt + kStages < ntiles) {
+            const int t0 = tok_begin + (tt + kStages) * kTile;
+            issue_tile_tc(st, &full[stage], a, b, kvh, t0, min(kTile, tok_end - t0), lane);
+        }
+        if (any) {
+            // exact tile maxima of every row and of the V scales
+#pragma unroll
+            for (int r = 0; r < RG; ++r) {
+                float v = sc[r];
+#pragma unroll
+                for (int m = 16; m >= 1; m >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, m));
+                if (lane == 0) s_red[warp * 16 + r] = v;
+            }
+            const unsigned vb = __reduce_max_sync(kFull, __float_as_uint(vs));
+            if (lane == 0) s_redv[warp] = vb;
+            __syncthreads();
+            const unsigned vmax = max(max(s_redv[0], s_redv[1]), max(s_redv[2], s_redv[3]));
+            const int ev_new = max(ev, (int)(vmax >> 23));
+            const float av = pow2i(ev - ev_new);
+            ev = ev_new;
+            vn = pow2i(127 - ev);
+            vlimit = ev >= 254 ? CUDART_INF_F : __uint_as_float((uint32_t)(ev + 1) << 23);
+            float alpha[RG];
+#pragma unroll
+            for (int r = 0; r < RG; ++r) {
+                const float tmax = fmaxf(fmaxf(s_red[r], s_red[16 + r]),
+                                         fmaxf(s_red[32 + r], s_red[48 + r]));
+                const float mn = fmaxf(m_run[r], tmax);
+                alpha[r] = mn == -CUDART_INF_F ? 1.f : fast_exp2(m_run[r] - mn);
+                m_run[r] = mn;
+                l_run[r] *= alpha[r];
+            }
+            if (tt > 0) {
+                // O^T row (dimension tid): column n holds row n % RG
+                uint32_t ov[NCOL];
+#pragma unroll
+                for (int c = 0; c < NCOL; c += 16) tmem_ld16(t_lane + kColO + c, ov + c);
+                tmem_wait_ld();
+#pragma unroll
+                for (int n = 0; n < NCOL; ++n)
+                    ov[n] = __float_as_uint(__uint_as_float(ov[n]) * (alpha[n % RG] * av));
+#pragma unroll
+                for (int c = 0; c < NCOL; c += 16) tmem_st16(t_lane + kColO + c, ov + c);
+            }
+            __syncthreads();   // s_red is reused by the next rescale
+        }
+
+        // P' row of token tid at K position kpos: hi columns, then lo columns
+        const float vn_t = vs * vn;
+        uint32_t hv[RG / 2], lv[RG / 2];
+#pragma unroll
+        for (int r = 0; r < RG; r += 2) {
+            float p0 = fast_exp2(sc[r] - m_run[r]);
+            float p1 = fast_exp2(sc[r + 1] - m_run[r + 1]);
+            if (!full_tile) {
+                p0 = sc[r] == -CUDART_INF_F ? 0.f : p0;
+                p1 = sc[r + 1] == -CUDART_INF_F ? 0.f : p1;
+            }
+            l_run[r] += p0;
+            l_run[r + 1] += p1;
+            float x0 = p0 * vn_t, x1 = p1 * vn_t;
+            if (!full_tile) {
+                x0 = p0 > 0.f ? x0 : 0.f;
+                x1 = p1 > 0.f ? x1 : 0.f;
+            }
+            hv[r / 2] = split_hi_lo<true>(x0, x1, true);
+            lv[r / 2] = split_hi_lo<true>(x0, x1, false);
+        }
+        {
+            uint8_t* rowp = s_pb + (kpos >> 3) * kCmRow + (kpos & 7) * 16;
+#pragma unroll
+            for (int g8 = 0; g8 < RG / 8; ++g8) {
+                *reinterpret_cast<uint4*>(rowp + g8 * 128) =
+                    make_uint4(hv[4 * g8], hv[4 * g8 + 1], hv[4 * g8 + 2], hv[4 * g8 + 3]);
+                *reinterpret_cast<uint4*>(rowp + (RG / 8 + g8) * 128) =
+                    make_uint4(lv[4 * g8], lv[4 * g8 + 1], lv[4 * g8 + 2], lv[4 * g8 + 3]);
+            }
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // 4. O^T += V^T P'
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                umma_f16_ts(tmem + kColO, tmem + 8 * j,
+                            smem_desc(s_pb + 2 * j * kCmRow, kCmRow, 128), kIdescO,
+                            (tt > 0 || j > 0) ? 1u : 0u);
+            umma_commit(bar_o);
+        }
+    }
+
+    // ---- epilogue: O rows into shared memory, l summed over the CTA
+    bool ok = !aborted && mbar_wait_bounded(bar_o, (uint32_t)((ntiles - 1) & 1), kSpinsTc);
+    tc_fence_after();
+    const int nrows = min(RG, a.G - rg * RG);
+    float* sO = reinterpret_cast<float*>(ring);          // [RG][128]
+    if (ok) {
+        uint32_t ov[NCOL];
+#pragma unroll
+        for (int c = 0; c < NCOL; c += 16) tmem_ld16(t_lane + kColO + c, ov + c);
+        tmem_wait_ld();
+        const float vback = pow2i(ev - 127);
+#pragma unroll
+        for (int r = 0; r < RG; ++r)
+            sO[r * kHeadDim + tid] = (__uint_as_float(ov[r]) + __uint_as_float(ov[RG + r])) * vback;
+#pragma unroll
+        for (int r = 0; r < RG; ++r) {
+            float l = l_run[r];
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) l += __shfl_xor_sync(kFull, l, m);
+            if (lane == 0) s_l[warp * 16 + r] = l;
+        }
+    } else if (tid == 0) {
+        report_error(a.err, TQ_ERR_TIMEOUT, kErrWaitTile);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+    if (!ok) return;
+
+    const int64_t unit = ((int64_t)b * gridDim.y + blockIdx.y);
+    const int64_t part = unit * a.max_splits + split;
+    const float rs = 0.08838834764831845f;
+    for (int rr = warp; rr < nrows; rr += 4) {
+        const float M = m_run[rr];
+        const float Lsum = s_l[rr] + s_l[16 + rr] + s_l[32 + rr] + s_l[48 + rr];
+        float x[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = sO[rr * kHeadDim + 4 * lane + e];
+        const int R = rg * RG + rr;
+        const int tq = R / a.group;
+        const int h = kvh * a.group + (R - tq * a.group);
+        if (nsplit == 1) {
+            const float inv = 1.f / Lsum;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) x[e] *= inv;
+            fwht128_lane(x, lane);
+            *reinterpret_cast<float4*>(a.out + (((int64_t)b * a.q_len + tq) * a.num_q_heads + h) *
+                                                   kHeadDim + 4 * lane) =
+                make_float4(x[0] * rs, x[1] * rs, x[2] * rs, x[3] * rs);
+        } else {
+            *reinterpret_cast<float4*>(a.ws_o + (part * RG + rr) * kHeadDim + 4 * lane) =
+                make_float4(x[0], x[1], x[2], x[3]);
+            if (lane == 0) a.ws_ml[part * RG + rr] = make_float2(M, Lsum);
+        }
+    }
+    if (nsplit == 1) return;
+
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const unsigned old = atomicInc(a.ws_cnt + unit, (unsigned)(nsplit - 1));
+        s_flag[1] = old == (unsigned)(nsplit - 1);
+    }
+    __syncthreads();
+    if (!s_flag[1]) return;
+    __threadfence();
+    for (int rr = warp; rr < nrows; rr += 4) {
+        const int64_t base = unit * a.max_splits;
+        float M = -CUDART_INF_F;
+        for (int sp = 0; sp < nsplit; ++sp)
+            M = fmaxf(M, __ldcg(a.ws_ml + (base + sp) * RG + rr).x);
+        float Lsum = 0.f;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int sp = 0; sp < nsplit; ++sp) {
+            const float2 ml = __ldcg(a.ws_ml + (base + sp) * RG + rr);
+            const float sc = ml.x == -CUDART_INF_F ? 0.f : exp2f(ml.x - M);
+            Lsum += sc * ml.y;
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(
+                a.ws_o + ((base + sp) * RG + rr) * kHeadDim) + lane);
+            acc[0] += sc * v.x;
+            acc[1] += sc * v.y;
+            acc[2] += sc * v.z;
+            acc[3] += sc * v.w;
+        }
+        const float inv = 1.f / Lsum;
+        float x[4] = {acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv};
+        fwht128_lane(x, lane);
+        const int R = rg * RG + rr;
+        const int tq = R / a.group;
+        const int h = kvh * a.group + (R - tq * a.group);
+        *reinterpret_cast<float4*>(a.out + (((int64_t)b * a.q_len + tq) * a.num_q_heads + h) *
+                                               kHeadDim + 4 * lane) =
+            make_float4(x[0] * rs, x[1] * rs, x[2] * rs, x[3] * rs);
+    }
+}
+
+template <int BITS, int NCOL>
+cudaError_t launch_tc(const TcArgs& a, dim3 grid, cudaStream_t stream)
+{
+    const size_t smem = 1024 + 2 * 256 * NCOL + (size_t)kStages * TcFmt<BITS>::kStage;
+    static int configured = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 31 || !(configured & (1 << dev))) {
+        e = cudaFuncSetAttribute(k_decode_tc<BITS, NCOL>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        if (dev < 31) configured |= 1 << dev;
+    }
+    k_decode_tc<BITS, NCOL><<<grid, kTcThreads, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// rows of one tensor-core CTA: 8 (N = 16) when G <= 8, else 16 (N = 32)
+int decode_tc_rows(int G) { return G <= 8 ? 8 : 16; }
+
+cudaError_t launch_decode_tc(const void* q, const tq_cache& c, int64_t block_bytes,
+                             const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                             int batch, int q_len, int num_q_heads, int max_seq_len, float* out,
+                             void* workspace, int split_tokens, cudaStream_t stream)
+{
+    TcArgs a{};
+    a.q = static_cast<const uint16_t*>(q);
+    a.kp = static_cast<const uint8_t*>(c.k_pages);
+    a.vp = static_cast<const uint8_t*>(c.v_pages);
+    a.page_table = page_table;
+    a.seq_lens = seq_lens;
+    a.out = out;
+    a.err = c.dev_error;
+    a.block_bytes = block_bytes;
+    a.max_pages = max_pages;
+    a.num_pages = c.num_pages;
+    a.num_kv_heads = c.num_kv_heads;
+    a.num_q_heads = num_q_heads;
+    a.group = num_q_heads / c.num_kv_heads;
+    a.q_len = q_len;
+    a.G = q_len * a.group;
+    const int rows = decode_tc_rows(a.G);
+    a.R = (a.G + rows - 1) / rows;
+    a.page_size = c.page_size;
+    a.split_tokens = split_tokens;
+    a.max_splits = (max_seq_len + split_tokens - 1) / split_tokens;
+    a.max_seq_len = max_seq_len;
+    if (a.max_splits > 1) {
+        const int64_t units = (int64_t)batch * c.num_kv_heads * a.R;
+        const int64_t cnt = ((units * 4 + 255) / 256) * 256;
+        const int64_t ml = ((units * a.max_splits * rows * 8 + 255) / 256) * 256;
+        uint8_t* w = static_cast<uint8_t*>(workspace);
+        a.ws_cnt = reinterpret_cast<uint32_t*>(w);
+        a.ws_ml = reinterpret_cast<float2*>(w + cnt);
+        a.ws_o = reinterpret_cast<float*>(w + cnt + ml);
+    }
+    const dim3 grid((unsigned)a.max_splits, (unsigned)(c.num_kv_heads * a.R), (unsigned)batch);
+#define TQ_TC(B) \
+    return rows == 8 ? launch_tc<B, 16>(a, grid, stream) : launch_tc<B, 32>(a, grid, stream)
+    switch (c.format) {
+    case 2: TQ_TC(2);
+    case 3: TQ_TC(3);
+    case 4: TQ_TC(4);
+    case 8: TQ_TC(8);
+    default: return cudaErrorInvalidValue;
+    }
+#undef TQ_TC
+}
+
+}  // namespace tq

@@ -110,7 +110,8 @@ def check_close(got: np.ndarray, ref: np.ndarray, what: str = "") -> dict:
 
 
 def gpu_rows(cache: tq.Cache, slots: np.ndarray, P: int, fmt: int):
-    """Packed code bytes and fp32 scales of K and V at `slots` (host copy)."""
+    """K packed rows, V offset-binary values (read from the dim-major V
+    block) and the fp32 scales of K and V at `slots` (host copy)."""
     pages = torch.as_tensor(slots // P, device="cuda")
     offs = slots % P
     kb = cache.k_pages[pages].cpu().numpy()
@@ -118,23 +119,27 @@ def gpu_rows(cache: tq.Cache, slots: np.ndarray, P: int, fmt: int):
     cb = 128 * fmt // 8
     idx = np.arange(len(slots))
     kc = np.stack([kb[i, :, offs[i] * cb:(offs[i] + 1) * cb] for i in idx])
-    vc = np.stack([vb[i, :, offs[i] * cb:(offs[i] + 1) * cb] for i in idx])
+    vbits = np.unpackbits(vb[:, :, :P * cb], axis=-1, bitorder="little")
+    vbits = vbits.reshape(len(slots), vb.shape[1], 128, P, fmt)[idx, :, :, offs]
+    vu = (vbits * (1 << np.arange(fmt))).sum(-1)
     so = P * cb
     ks = np.stack([kb[i, :, so + 4 * offs[i]:so + 4 * offs[i] + 4] for i in idx]).view(np.float32)
     vs = np.stack([vb[i, :, so + 4 * offs[i]:so + 4 * offs[i] + 4] for i in idx]).view(np.float32)
-    return kc, vc, ks[..., 0], vs[..., 0]
+    return kc, vu, ks[..., 0], vs[..., 0]
 
 
 def oracle_rows(w: W.Workload, slots: np.ndarray, fmt: int):
     k, v = w.kv_for_slots(slots)
     n, H = len(slots), w.num_kv_heads
     cb = 128 * fmt // 8
+    L = (1 << (fmt - 1)) - 1
     kc = np.zeros((n, H, cb), np.uint8)
-    vc = np.zeros_like(kc)
+    vu = np.zeros((n, H, 128), np.int64)
     ks = np.zeros((n, H), np.float32)
     vs = np.zeros_like(ks)
     for i in range(n):
         for h in range(H):
             kc[i, h], ks[i, h] = oracle.quantize_vector(k[i, h], fmt)
-            vc[i, h], vs[i, h] = oracle.quantize_vector(v[i, h], fmt)
-    return kc, vc, ks, vs
+            codes, vs[i, h] = oracle.quantize_rotated(oracle.rotate_f32(v[i, h]), fmt)
+            vu[i, h] = codes + L
+    return kc, vu, ks, vs

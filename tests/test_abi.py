@@ -116,11 +116,11 @@ def test_decode_validation():
 def test_workspace_size():
     c = desc()
     ws = tq.lib().tq_decode_workspace_size
-    # one split (<= 512 tokens with 16-token pages): no workspace
-    assert ws(8, 1, 32, 512, ctypes.byref(c)) == 0
-    n = ws(8, 1, 32, 4096, ctypes.byref(c))
-    # 8 splits x 64 (seq, kv head) units x 8 rows x (128 + 2) floats + counters
-    assert n >= 8 * 64 * 8 * 130 * 4 and n < 8 * 64 * 8 * 130 * 4 + 4096
+    # one split (<= 2048 tokens with 16-token pages): no workspace
+    assert ws(8, 1, 32, 2048, ctypes.byref(c)) == 0
+    n = ws(8, 1, 32, 8192, ctypes.byref(c))
+    # 4 splits x 64 (seq, kv head) units x 8 rows x (128 + 2) floats + counters
+    assert n >= 4 * 64 * 8 * 130 * 4 and n < 4 * 64 * 8 * 130 * 4 + 4096
     assert ws(8, 1, 30, 4096, ctypes.byref(c)) == 0   # invalid
     c64 = desc(P=64)
     assert ws(4, 1, 40, 131072, ctypes.byref(c64)) >= 4 * 8 * 128 * 8 * 130 * 4

@@ -25,8 +25,8 @@ TURBO = (2, 3, 4, 8)
 
 
 def small(fmt, **kw):
-    base = dict(batch=3, num_q_heads=8, num_kv_heads=2, page_size=16, q_len=1,
-                seq_lens=(1300, 37, 513), fmt=fmt, seed=11 + fmt)
+    base = dict(num_q_heads=8, num_kv_heads=2, page_size=16, q_len=1,
+                seq_lens=(2600, 37, 2049), fmt=fmt, seed=11 + fmt)
     base.update(kw)
     return W.custom(**base)
 
@@ -86,7 +86,7 @@ def test_quantize_full_size_sampled(name, fmt):
     got = gpu_rows(cache, s, w.page_size, fmt)
     ref = oracle_rows(w, s, fmt)
     for a, b in zip(got, ref):
-        assert np.array_equal(a.view(np.uint8), b.view(np.uint8))
+        assert a.shape == b.shape and np.array_equal(np.asarray(a), np.asarray(b))
     assert cache.read_error() == 0
 
 
@@ -95,10 +95,10 @@ def test_quantize_full_size_sampled(name, fmt):
 @pytest.mark.parametrize("q_len,Hq,Hkv", [(1, 8, 2), (1, 10, 2), (4, 8, 2), (3, 6, 1),
                                           (1, 16, 1), (8, 64, 8)])
 def test_decode_small(fmt, q_len, Hq, Hkv):
-    """Ragged lengths (1300 = 2 splits + tail, 37 < one tile, 513 = one
+    """Ragged lengths (2600 = 2 splits + tail, 37 < one tile, 2049 = one
     token past a split), 1-8 query rows per kv head up to 16 and 64."""
     w = small(fmt, q_len=q_len, num_q_heads=Hq, num_kv_heads=Hkv,
-              seq_lens=(1300, 37 + q_len, 513))
+              seq_lens=(2600, 37 + q_len, 2049))
     cache = gpu_fill(w, fmt)
     got = gpu_decode(w, fmt, cache)
     ref = oracle_decode(w, fmt, np.arange(w.batch))
@@ -141,7 +141,7 @@ def test_decode_configs(name, fmt, seqs):
 @pytest.mark.parametrize("fmt", (4, 16))
 def test_batch_invariance(fmt):
     """A sequence's output is bit-identical alone and inside a batch."""
-    w = small(fmt, seq_lens=(1300, 37, 513, 2049), batch=4)
+    w = small(fmt, seq_lens=(2600, 37, 2049, 4100))
     cache = gpu_fill(w, fmt)
     full = gpu_decode(w, fmt, cache)
     q = w.queries()
@@ -169,15 +169,15 @@ def test_page_permutation_invariance():
 def test_shared_prefix_equals_private_copies():
     """Sequences reading one physical copy of a prefix give the same bits as
     sequences holding private copies of the same prefix values."""
-    shared = W.custom(batch=3, seq_lens=(600, 900, 1100), q_len=4, num_q_heads=8,
-                      num_kv_heads=2, shared_prefix_seqs=3, shared_prefix_tokens=512,
+    shared = W.custom(seq_lens=(2600, 3000, 2300), q_len=4, num_q_heads=8,
+                      num_kv_heads=2, shared_prefix_seqs=3, shared_prefix_tokens=1024,
                       permute_pages=False, fmt=4, seed=9)
     cache = gpu_fill(shared, 4)
     out = gpu_decode(shared, 4, cache)
     # private layout: copy the prefix pages for sequences 1 and 2
     from quantized_paged_kv_tq_b200 import tq as T
     P = shared.page_size
-    npre = 512 // P
+    npre = 1024 // P
     extra = 2 * npre
     c2 = T.Cache(4, shared.num_pages + extra, 2, P)
     c2.k_pages[:shared.num_pages] = cache.k_pages
@@ -202,9 +202,9 @@ def test_append_order_independence():
 
 
 def test_causal_last_split_fully_masked_rows():
-    """seq_len 514 with q_len 4: the second split holds keys 512-513 only,
-    which rows t = 0, 1 must not see (their partial is empty)."""
-    w = small(4, q_len=4, seq_lens=(514, 516), batch=2)
+    """seq_len 2050 with q_len 4: the second split holds keys 2048-2049
+    only, which rows t = 0, 1 must not see (their partial is empty)."""
+    w = small(4, q_len=4, seq_lens=(2050, 2052))
     cache = gpu_fill(w, 4)
     check_close(gpu_decode(w, 4, cache), oracle_decode(w, 4, np.arange(2)))
 

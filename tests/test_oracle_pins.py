@@ -236,12 +236,23 @@ def _fill(w, fmt):
     return kp, vp
 
 
-def _dequant_numpy(pool, fmt, page, kvh, off, P, d=128):
-    """Rotated dequantised row via numpy's little-endian unpackbits."""
+def _unpack_u(pool, fmt, page, kvh, off, P, dim_major, d=128):
+    """Offset-binary values u of one token via numpy's little-endian
+    unpackbits: K blocks hold token rows, V blocks dimension rows."""
     cb = d * fmt // 8
     blk = pool[page, kvh]
-    bits = np.unpackbits(blk[off * cb:(off + 1) * cb], bitorder="little")
-    u = (bits.reshape(d, fmt) * (1 << np.arange(fmt))).sum(1)
+    if dim_major:
+        bits = np.unpackbits(blk[:P * cb], bitorder="little").reshape(d, P, fmt)[:, off]
+    else:
+        bits = np.unpackbits(blk[off * cb:(off + 1) * cb], bitorder="little").reshape(d, fmt)
+    return (bits * (1 << np.arange(fmt))).sum(1)
+
+
+def _dequant_numpy(pool, fmt, page, kvh, off, P, dim_major=False, d=128):
+    """Rotated dequantised row (code * s / L)."""
+    cb = d * fmt // 8
+    blk = pool[page, kvh]
+    u = _unpack_u(pool, fmt, page, kvh, off, P, dim_major, d)
     s = blk[P * cb + 4 * off:P * cb + 4 * off + 4].view(np.float32)[0]
     L = Lof(fmt)
     return (u - L) * float(s) / L
@@ -274,7 +285,7 @@ def test_paged_decode_matches_sdpa(fmt, q_len):
                     V[j] = W.bf16_bits_to_f32(vp[page, kvh, off])
                 else:
                     K[j] = H @ _dequant_numpy(kp, fmt, page, kvh, off, P)
-                    V[j] = H @ _dequant_numpy(vp, fmt, page, kvh, off, P)
+                    V[j] = H @ _dequant_numpy(vp, fmt, page, kvh, off, P, dim_major=True)
             qr = W.bf16_bits_to_f32(q[b, :, h]).astype(np.float64)
             ref = _sdpa(qr, K, V, [n - q_len + t for t in range(q_len)])
             assert np.max(np.abs(out[b, :, h] - ref)) < 1e-11
@@ -340,25 +351,34 @@ def test_causal_rows_equal_shorter_single_token_decode(fmt):
         assert np.array_equal(single[:, 0], out[:, t])
 
 
-def test_quantize_append_layout_and_skip():
-    """Appended rows land at block (page, head), row `offset`, scale after
-    the codes; slot -1 writes nothing."""
-    rng = np.random.default_rng(50)
-    k = rand_bf16(rng, (3, 2, 128))
-    v = rand_bf16(rng, (3, 2, 128))
-    kp = np.zeros((4, 2, oracle.block_bytes(4, 128, 16)), np.uint8)
+@pytest.mark.parametrize("bits,P", [(4, 16), (3, 16), (2, 32), (8, 64), (3, 64)])
+def test_quantize_append_layout_and_skip(bits, P):
+    """K rows land at block (page, head), token row `offset`; V codes land
+    dim-major (dimension i's row holds every token's field i); scales follow
+    the codes; slot -1 writes nothing; other tokens' fields are untouched."""
+    rng = np.random.default_rng(50 + bits)
+    k = rand_bf16(rng, (4, 2, 128))
+    v = rand_bf16(rng, (4, 2, 128))
+    cb = 128 * bits // 8
+    kp = np.zeros((4, 2, oracle.block_bytes(bits, 128, P)), np.uint8)
     vp = np.zeros_like(kp)
-    oracle.quantize_append(k, v, np.array([5, -1, 16 * 3 + 15]), 4, 16, kp, vp)
-    for t, (page, off) in ((0, (0, 5)), (2, (3, 15))):
+    slots = np.array([5, -1, P * 3 + P - 1, 6])
+    oracle.quantize_append(k, v, slots, bits, P, kp, vp)
+    L = Lof(bits)
+    for t, (page, off) in ((0, (0, 5)), (2, (3, P - 1)), (3, (0, 6))):
         for h in range(2):
-            pk, sk = oracle.quantize_vector(k[t, h], 4)
-            pv, sv = oracle.quantize_vector(v[t, h], 4)
-            assert np.array_equal(kp[page, h, off * 64:(off + 1) * 64], pk)
-            assert np.array_equal(vp[page, h, off * 64:(off + 1) * 64], pv)
-            assert kp[page, h, 1024 + 4 * off:1028 + 4 * off].view(np.float32)[0] == sk
-            assert vp[page, h, 1024 + 4 * off:1028 + 4 * off].view(np.float32)[0] == sv
-    written = {(0, 5), (3, 15)}
+            pk, sk = oracle.quantize_vector(k[t, h], bits)
+            yv = oracle.rotate_f32(v[t, h])
+            cv, sv = oracle.quantize_rotated(yv, bits)
+            assert np.array_equal(kp[page, h, off * cb:(off + 1) * cb], pk)
+            assert np.array_equal(_unpack_u(vp, bits, page, h, off, P, True), cv + L)
+            so = P * cb + 4 * off
+            assert kp[page, h, so:so + 4].view(np.float32)[0] == sk
+            assert vp[page, h, so:so + 4].view(np.float32)[0] == sv
+    written = {(0, 5), (3, P - 1), (0, 6)}
     for page in range(4):
-        for off in range(16):
+        for off in range(P):
             if (page, off) not in written:
-                assert not kp[page, :, off * 64:(off + 1) * 64].any()
+                assert not kp[page, :, off * cb:(off + 1) * cb].any()
+                for h in range(2):
+                    assert not _unpack_u(vp, bits, page, h, off, P, True).any()
