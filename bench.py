@@ -69,12 +69,23 @@ def measured_peaks():
         return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
 
 
+DECODE_SOURCES = ("decode.cu", "decode_tc.cu", "tq_device.cuh")
+
+
+def decode_sources_sha256() -> str:
+    """sha256 over the decode kernels' sources, in DECODE_SOURCES order."""
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "quantized_paged_kv_tq_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def profiled_traffic(kernel: str):
     """dram read+write bytes per launch recorded in profiles/<kernel>*.txt,
-    valid only while decode.cu is unchanged (its sha256 is recorded too)."""
-    src = os.path.join(ROOT, "quantized_paged_kv_tq_b200", "csrc", "decode.cu")
-    with open(src, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()
+    valid only while the decode sources are unchanged (their sha256 is
+    recorded as decode_src_sha256)."""
+    sha = decode_sources_sha256()
     pdir = os.path.join(ROOT, "profiles")
     if not os.path.isdir(pdir):
         return None
@@ -87,7 +98,7 @@ def profiled_traffic(kernel: str):
                 if ":" in line:
                     k, v = line.split(":", 1)
                     vals[k.strip()] = v.strip()
-        if vals.get("decode_cu_sha256") == sha and "traffic_bytes_per_launch" in vals:
+        if vals.get("decode_src_sha256") == sha and "traffic_bytes_per_launch" in vals:
             return float(vals["traffic_bytes_per_launch"])
     return None
 

@@ -872,7 +872,7 @@ int decode_split_tokens(int page_size)
 }
 
 
-int decode_tc_rows(int G);
+int decode_tc_rows(int format, int G);
 cudaError_t launch_decode_tc(const void* q, const tq_cache& c, int64_t block_bytes,
                              const int32_t* page_table, int max_pages, const int32_t* seq_lens,
                              int batch, int q_len, int num_q_heads, int max_seq_len, float* out,
@@ -880,7 +880,10 @@ cudaError_t launch_decode_tc(const void* q, const tq_cache& c, int64_t block_byt
 
 // Query rows per CTA: the tensor-core kernel (turbo formats) takes 8 or 16,
 // the warp-MMA kernel (bf16) 8.
-int decode_rows_per_cta(int format, int G) { return format == 16 ? kRowsPerCta : decode_tc_rows(G); }
+int decode_rows_per_cta(int format, int G)
+{
+    return format == 16 ? kRowsPerCta : decode_tc_rows(format, G);
+}
 
 int decode_row_groups(int format, int G)
 {

@@ -41,7 +41,7 @@ constexpr int kStages = 2;
 constexpr uint32_t kTmemCols = 128;      // A: 64 columns, S: N, O: N (N <= 32)
 constexpr float kLog2eTc = 1.4426950408889634f;
 constexpr float kLazyTc = 8.f;
-constexpr uint32_t kSpinsTc = 1u << 24;
+constexpr uint32_t kPollsTc = 1u << 16;       // x 20 us sleeping polls
 constexpr uint32_t kMagicTc = 0x64006400u;
 
 struct TcArgs {
@@ -283,12 +283,92 @@ __device__ __forceinline__ void issue_tile_tc(uint8_t* stage, uint64_t* bar, con
     }
 }
 
-template <int BITS, int NCOL>
+// Split epilogue shared by the tensor-core kernels.  sO: the split's
+// un-normalised output rows [RG][128] (rotated domain); s_l: per-warp partial
+// row sums [4][16]; m_run: row maxima (log2 units).  A split that is the whole
+// sequence normalises, rotates back and writes; otherwise the partial goes to
+// the workspace and the last split CTA of the unit (atomic ticket) merges.
+template <int RG>
+__device__ __forceinline__ void tc_finish(const TcArgs& a, const float* sO, const float* s_l,
+                                          const float* m_run, int* s_flag, int b, int kvh, int rg,
+                                          int split, int nsplit, int nrows, int warp, int lane,
+                                          int tid)
+{
+    const int64_t unit = ((int64_t)b * gridDim.y + blockIdx.y);
+    const int64_t part = unit * a.max_splits + split;
+    const float rs = 0.08838834764831845f;
+    for (int rr = warp; rr < nrows; rr += 4) {
+        const float M = m_run[rr];
+        const float Lsum = s_l[rr] + s_l[16 + rr] + s_l[32 + rr] + s_l[48 + rr];
+        float x[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = sO[rr * kHeadDim + 4 * lane + e];
+        const int R = rg * RG + rr;
+        const int tq = R / a.group;
+        const int h = kvh * a.group + (R - tq * a.group);
+        if (nsplit == 1) {
+            const float inv = 1.f / Lsum;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) x[e] *= inv;
+            fwht128_lane(x, lane);
+            *reinterpret_cast<float4*>(a.out + (((int64_t)b * a.q_len + tq) * a.num_q_heads + h) *
+                                                   kHeadDim + 4 * lane) =
+                make_float4(x[0] * rs, x[1] * rs, x[2] * rs, x[3] * rs);
+        } else {
+            *reinterpret_cast<float4*>(a.ws_o + (part * RG + rr) * kHeadDim + 4 * lane) =
+                make_float4(x[0], x[1], x[2], x[3]);
+            if (lane == 0) a.ws_ml[part * RG + rr] = make_float2(M, Lsum);
+        }
+    }
+    if (nsplit == 1) return;
+
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const unsigned old = atomicInc(a.ws_cnt + unit, (unsigned)(nsplit - 1));
+        s_flag[1] = old == (unsigned)(nsplit - 1);
+    }
+    __syncthreads();
+    if (!s_flag[1]) return;
+    __threadfence();
+    for (int rr = warp; rr < nrows; rr += 4) {
+        const int64_t base = unit * a.max_splits;
+        float M = -CUDART_INF_F;
+        for (int sp = 0; sp < nsplit; ++sp)
+            M = fmaxf(M, __ldcg(a.ws_ml + (base + sp) * RG + rr).x);
+        float Lsum = 0.f;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int sp = 0; sp < nsplit; ++sp) {
+            const float2 ml = __ldcg(a.ws_ml + (base + sp) * RG + rr);
+            const float sc = ml.x == -CUDART_INF_F ? 0.f : exp2f(ml.x - M);
+            Lsum += sc * ml.y;
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(
+                a.ws_o + ((base + sp) * RG + rr) * kHeadDim) + lane);
+            acc[0] += sc * v.x;
+            acc[1] += sc * v.y;
+            acc[2] += sc * v.z;
+            acc[3] += sc * v.w;
+        }
+        const float inv = 1.f / Lsum;
+        float x[4] = {acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv};
+        fwht128_lane(x, lane);
+        const int R = rg * RG + rr;
+        const int tq = R / a.group;
+        const int h = kvh * a.group + (R - tq * a.group);
+        *reinterpret_cast<float4*>(a.out + (((int64_t)b * a.q_len + tq) * a.num_q_heads + h) *
+                                               kHeadDim + 4 * lane) =
+            make_float4(x[0] * rs, x[1] * rs, x[2] * rs, x[3] * rs);
+    }
+}
+
+template <int BITS, int RG>
 __global__ void __launch_bounds__(kTcThreads, 4)
 k_decode_tc(const TcArgs a)
 {
     using F = TcFmt<BITS>;
-    constexpr int RG = NCOL / 2;              // query rows per CTA
+    // RG query rows per CTA; operand columns: hi parts [0, RG), lo parts
+    // [RG, 2 RG), zero padding up to NCOL (the MMA needs N >= 16)
+    constexpr int NCOL = 2 * RG < 16 ? 16 : 2 * RG;
     constexpr uint32_t kColS = 64, kColO = 64 + NCOL;
     // instruction descriptors: f32 accumulate, f16 operands, M = 128, N = NCOL;
     // B K-major (Q') for S, B MN-major (P') for O
@@ -396,7 +476,7 @@ k_decode_tc(const TcArgs a)
         __half* qb = reinterpret_cast<__half*>(s_qb);
 #pragma unroll
         for (int n = 0; n < NCOL; ++n) {
-            const float v = s_qf[(n % RG) * kHeadDim + dim];
+            const float v = n < 2 * RG ? s_qf[(n % RG) * kHeadDim + dim] : 0.f;
             const float hi = __half2float(__float2half_rn(v));
             const __half h = __float2half_rn(n < RG ? v : v - hi);
             const int cm = (k >> 3) * (NCOL / 8) + (n >> 3);
@@ -411,8 +491,18 @@ k_decode_tc(const TcArgs a)
         const int R = rg * RG + r;
         lim[r] = R < a.G ? seq_len - a.q_len + R / a.group : -1;
     }
+    __syncthreads();   // the q staging (aliasing the P' buffer) is consumed
+    if (2 * RG < NCOL) {
+        // zero padding columns of the P' operand, written once
+        uint8_t* rowp = s_pb + (tid >> 3) * kCmRow + (tid & 7) * 16;
+#pragma unroll
+        for (int ng = 2 * RG / 8; ng < NCOL / 8; ++ng)
+            *reinterpret_cast<uint4*>(rowp + ng * 128) = make_uint4(0u, 0u, 0u, 0u);
+    }
     fence_proxy_async_smem();
     __syncthreads();
+    const uint64_t desc_q = smem_desc(s_qb, kCmRow, 128);
+    const uint64_t desc_p = smem_desc(s_pb, kCmRow, 128);
 
     float m_run[RG], l_run[RG];
 #pragma unroll
@@ -432,8 +522,8 @@ k_decode_tc(const TcArgs a)
         const int stage = tt % kStages;
         uint8_t* st = ring + stage * F::kStage;
         const int tok0 = tok_begin + tt * kTile;
-        bool ok = mbar_wait_bounded(&full[stage], (uint32_t)((tt / kStages) & 1), kSpinsTc);
-        if (tt > 0) ok = ok && mbar_wait_bounded(bar_o, (uint32_t)((tt - 1) & 1), kSpinsTc);
+        bool ok = mbar_wait_sleep(&full[stage], (uint32_t)((tt / kStages) & 1), kPollsTc);
+        if (tt > 0) ok = ok && mbar_wait_sleep(bar_o, (uint32_t)((tt - 1) & 1), kPollsTc);
         tc_fence_after();
         if (!ok) atomicOr(&s_flag[0], 1);
 
@@ -456,11 +546,11 @@ k_decode_tc(const TcArgs a)
             tc_fence_after();
 #pragma unroll
             for (int j = 0; j < 8; ++j)
-                umma_f16_ts(tmem + kColS, tmem + 8 * j,
-                            smem_desc(s_qb + 2 * j * kCmRow, kCmRow, 128), kIdescS, j > 0);
+                umma_f16_ts(tmem + kColS, tmem + 8 * j, desc_q + ((2 * j * kCmRow) >> 4), kIdescS,
+                            j > 0);
             umma_commit(bar_s);
         }
-        ok = mbar_wait_bounded(bar_s, (uint32_t)(tt & 1), kSpinsTc);
+        ok = mbar_wait_sleep(bar_s, (uint32_t)(tt & 1), kPollsTc);
         tc_fence_after();
         if (!ok) atomicOr(&s_flag[0], 1);
 
@@ -532,7 +622,9 @@ k_decode_tc(const TcArgs a)
 
         // P' row of token tid at K position kpos: hi columns, then lo columns
         const float vn_t = vs * vn;
-        uint32_t hv[RG / 2], lv[RG / 2];
+        uint32_t hl[RG];          // half2 pairs: hi parts [0, RG/2), lo parts [RG/2, RG)
+        uint32_t* hv = hl;
+        uint32_t* lv = hl + RG / 2;
 #pragma unroll
         for (int r = 0; r < RG; r += 2) {
             float p0 = fast_exp2(sc[r] - m_run[r]);
@@ -554,12 +646,9 @@ k_decode_tc(const TcArgs a)
         {
             uint8_t* rowp = s_pb + (kpos >> 3) * kCmRow + (kpos & 7) * 16;
 #pragma unroll
-            for (int g8 = 0; g8 < RG / 8; ++g8) {
-                *reinterpret_cast<uint4*>(rowp + g8 * 128) =
-                    make_uint4(hv[4 * g8], hv[4 * g8 + 1], hv[4 * g8 + 2], hv[4 * g8 + 3]);
-                *reinterpret_cast<uint4*>(rowp + (RG / 8 + g8) * 128) =
-                    make_uint4(lv[4 * g8], lv[4 * g8 + 1], lv[4 * g8 + 2], lv[4 * g8 + 3]);
-            }
+            for (int ng = 0; ng < 2 * RG / 8; ++ng)
+                *reinterpret_cast<uint4*>(rowp + ng * 128) =
+                    make_uint4(hl[4 * ng], hl[4 * ng + 1], hl[4 * ng + 2], hl[4 * ng + 3]);
         }
         tmem_wait_st();
         fence_proxy_async_smem();
@@ -571,15 +660,14 @@ k_decode_tc(const TcArgs a)
             tc_fence_after();
 #pragma unroll
             for (int j = 0; j < 8; ++j)
-                umma_f16_ts(tmem + kColO, tmem + 8 * j,
-                            smem_desc(s_pb + 2 * j * kCmRow, kCmRow, 128), kIdescO,
+                umma_f16_ts(tmem + kColO, tmem + 8 * j, desc_p + ((2 * j * kCmRow) >> 4), kIdescO,
                             (tt > 0 || j > 0) ? 1u : 0u);
             umma_commit(bar_o);
         }
     }
 
     // ---- epilogue: O rows into shared memory, l summed over the CTA
-    bool ok = !aborted && mbar_wait_bounded(bar_o, (uint32_t)((ntiles - 1) & 1), kSpinsTc);
+    bool ok = !aborted && mbar_wait_sleep(bar_o, (uint32_t)((ntiles - 1) & 1), kPollsTc);
     tc_fence_after();
     const int nrows = min(RG, a.G - rg * RG);
     float* sO = reinterpret_cast<float*>(ring);          // [RG][128]
@@ -610,95 +698,597 @@ k_decode_tc(const TcArgs a)
     }
     if (!ok) return;
 
-    const int64_t unit = ((int64_t)b * gridDim.y + blockIdx.y);
-    const int64_t part = unit * a.max_splits + split;
-    const float rs = 0.08838834764831845f;
-    for (int rr = warp; rr < nrows; rr += 4) {
-        const float M = m_run[rr];
-        const float Lsum = s_l[rr] + s_l[16 + rr] + s_l[32 + rr] + s_l[48 + rr];
-        float x[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = sO[rr * kHeadDim + 4 * lane + e];
-        const int R = rg * RG + rr;
-        const int tq = R / a.group;
-        const int h = kvh * a.group + (R - tq * a.group);
-        if (nsplit == 1) {
-            const float inv = 1.f / Lsum;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) x[e] *= inv;
-            fwht128_lane(x, lane);
-            *reinterpret_cast<float4*>(a.out + (((int64_t)b * a.q_len + tq) * a.num_q_heads + h) *
-                                                   kHeadDim + 4 * lane) =
-                make_float4(x[0] * rs, x[1] * rs, x[2] * rs, x[3] * rs);
-        } else {
-            *reinterpret_cast<float4*>(a.ws_o + (part * RG + rr) * kHeadDim + 4 * lane) =
-                make_float4(x[0], x[1], x[2], x[3]);
-            if (lane == 0) a.ws_ml[part * RG + rr] = make_float2(M, Lsum);
-        }
-    }
-    if (nsplit == 1) return;
+    tc_finish<RG>(a, sO, s_l, m_run, s_flag, b, kvh, rg, split, nsplit, nrows, warp, lane, tid);
+}
 
-    __syncthreads();
-    if (tid == 0) {
-        __threadfence();
-        const unsigned old = atomicInc(a.ws_cnt + unit, (unsigned)(nsplit - 1));
-        s_flag[1] = old == (unsigned)(nsplit - 1);
-    }
-    __syncthreads();
-    if (!s_flag[1]) return;
-    __threadfence();
-    for (int rr = warp; rr < nrows; rr += 4) {
-        const int64_t base = unit * a.max_splits;
-        float M = -CUDART_INF_F;
-        for (int sp = 0; sp < nsplit; ++sp)
-            M = fmaxf(M, __ldcg(a.ws_ml + (base + sp) * RG + rr).x);
-        float Lsum = 0.f;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int sp = 0; sp < nsplit; ++sp) {
-            const float2 ml = __ldcg(a.ws_ml + (base + sp) * RG + rr);
-            const float sc = ml.x == -CUDART_INF_F ? 0.f : exp2f(ml.x - M);
-            Lsum += sc * ml.y;
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(
-                a.ws_o + ((base + sp) * RG + rr) * kHeadDim) + lane);
-            acc[0] += sc * v.x;
-            acc[1] += sc * v.y;
-            acc[2] += sc * v.z;
-            acc[3] += sc * v.w;
-        }
-        const float inv = 1.f / Lsum;
-        float x[4] = {acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv};
-        fwht128_lane(x, lane);
-        const int R = rg * RG + rr;
-        const int tq = R / a.group;
-        const int h = kvh * a.group + (R - tq * a.group);
-        *reinterpret_cast<float4*>(a.out + (((int64_t)b * a.q_len + tq) * a.num_q_heads + h) *
-                                               kHeadDim + 4 * lane) =
-            make_float4(x[0] * rs, x[1] * rs, x[2] * rs, x[3] * rs);
+// ===================================================================
+// Integer tensor-core variant (kind::i8) for 2-, 4- and 8-bit codes.
+//
+//   S = K q''  A: K codes as unsigned bytes u (tensor memory, 32 columns);
+//              B: the scaled query q'' = rint(q' 2^s) as three balanced
+//              signed byte digits per row (column 4r + d); the accumulator
+//              starts at -L * sum(digits) so it holds sum (u - L) q'' exactly.
+//   O^T += V^T P''  A: V codes as signed bytes u - L (dim-major rows);
+//              B: P'' = rint(p s_v / L 2^(127 - ev) 2^22) as four unsigned
+//              byte digits per row.  O stays an exact int32 sum in tensor
+//              memory until the softmax rescales (rare) or the split ends,
+//              then it is folded into fp32 registers.
+// ===================================================================
+template <int BITS>
+struct I8Fmt {
+    static constexpr int CB = 16 * BITS;
+    static constexpr int L = (1 << (BITS - 1)) - 1;
+    static constexpr int kStage = 2 * kTile * (CB + 4);
+};
+
+// K position k of the byte operands -> dimension (K) or token (V)
+template <int BITS>
+__device__ __forceinline__ int perm_i8(int k)
+{
+    if constexpr (BITS == 4) return 8 * (k >> 3) + 2 * (k & 3) + ((k & 7) >> 2);
+    if constexpr (BITS == 2) return 16 * (k >> 4) + 4 * (k & 3) + ((k & 15) >> 2);
+    return k;
+}
+template <int BITS>
+__device__ __forceinline__ int perm_i8_inv(int i)
+{
+    if constexpr (BITS == 4) return 8 * (i >> 3) + ((i & 7) >> 1) + 4 * (i & 1);
+    if constexpr (BITS == 2) return 16 * (i >> 4) + 4 * (i & 3) + ((i & 15) >> 2);
+    return i;
+}
+
+// one word of codes -> unsigned bytes (u) in K-position order
+template <int BITS>
+__device__ __forceinline__ void u8_of(uint32_t w, uint32_t* o)
+{
+    if constexpr (BITS == 4) {
+        o[0] = w & 0x0F0F0F0Fu;
+        o[1] = (w >> 4) & 0x0F0F0F0Fu;
+    } else if constexpr (BITS == 2) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) o[j] = (w >> (2 * j)) & 0x03030303u;
+    } else {
+        o[0] = w;
     }
 }
 
-template <int BITS, int NCOL>
+// bytes u -> signed bytes u - L, byte-wise without carries
+template <int BITS>
+__device__ __forceinline__ uint32_t s8_of(uint32_t u)
+{
+    if constexpr (BITS == 8) {
+        // (u + 129) mod 256 per byte
+        const uint32_t t = (u & 0x7F7F7F7Fu) + 0x01010101u;
+        uint32_t r;
+        asm("lop3.b32 %0, %1, %2, %3, 0xD2;" : "=r"(r) : "r"(t), "r"(u), "r"(0x80808080u));
+        return r;   // t ^ (~u & 0x80..): adds 128 + (u & 128) without a carry out
+    } else {
+        constexpr uint32_t Lb = (uint32_t)I8Fmt<BITS>::L * 0x01010101u;
+        return ((u | 0x80808080u) - Lb) ^ 0x80808080u;
+    }
+}
+
+template <int BITS>
+__device__ __forceinline__ void k_row_to_tmem_u8(const uint8_t* row, uint32_t taddr)
+{
+    uint32_t o[16];
+    if constexpr (BITS == 4) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint4 a = *reinterpret_cast<const uint4*>(row + 32 * h);
+            const uint4 b = *reinterpret_cast<const uint4*>(row + 32 * h + 16);
+            u8_of<4>(a.x, o); u8_of<4>(a.y, o + 2); u8_of<4>(a.z, o + 4); u8_of<4>(a.w, o + 6);
+            u8_of<4>(b.x, o + 8); u8_of<4>(b.y, o + 10); u8_of<4>(b.z, o + 12); u8_of<4>(b.w, o + 14);
+            tmem_st16(taddr + 16 * h, o);
+        }
+    } else if constexpr (BITS == 2) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint4 a = *reinterpret_cast<const uint4*>(row + 16 * h);
+            u8_of<2>(a.x, o); u8_of<2>(a.y, o + 4); u8_of<2>(a.z, o + 8); u8_of<2>(a.w, o + 12);
+            tmem_st16(taddr + 16 * h, o);
+        }
+    } else {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 a = *reinterpret_cast<const uint4*>(row + 64 * h + 16 * q);
+                o[4 * q] = a.x; o[4 * q + 1] = a.y; o[4 * q + 2] = a.z; o[4 * q + 3] = a.w;
+            }
+            tmem_st16(taddr + 16 * h, o);
+        }
+    }
+}
+
+// V codes of dimension `dim` for the tile's 128 tokens -> 32 words of
+// signed bytes in K-position order (registers; stored once the previous
+// PV product has drained).
+template <int BITS>
+__device__ __forceinline__ void v_col_s8(const uint8_t* vblk0, int64_t bb, int P, int dim,
+                                         uint32_t* o)
+{
+    // 32 tokens per chunk: 16 bytes (4-bit), 8 bytes (2-bit), 32 bytes (8-bit)
+    const int row_bytes = P * BITS / 8;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int t0 = 32 * q;
+        const int pg = t0 / P, in = t0 % P;
+        const uint8_t* row = vblk0 + pg * bb + (int64_t)dim * row_bytes;
+        uint32_t w[8];
+        if constexpr (BITS == 4) {
+            if (P >= 32) {
+                const uint4 x = *reinterpret_cast<const uint4*>(row + in / 2);
+                w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
+            } else {
+                const uint2 x = *reinterpret_cast<const uint2*>(row);
+                const uint2 y = *reinterpret_cast<const uint2*>(row + bb);
+                w[0] = x.x; w[1] = x.y; w[2] = y.x; w[3] = y.y;
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint32_t u[2];
+                u8_of<4>(w[i], u);
+                o[8 * q + 2 * i] = s8_of<4>(u[0]);
+                o[8 * q + 2 * i + 1] = s8_of<4>(u[1]);
+            }
+        } else if constexpr (BITS == 2) {
+            if (P >= 32) {
+                const uint2 x = *reinterpret_cast<const uint2*>(row + in / 4);
+                w[0] = x.x; w[1] = x.y;
+            } else {
+                w[0] = *reinterpret_cast<const uint32_t*>(row);
+                w[1] = *reinterpret_cast<const uint32_t*>(row + bb);
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                uint32_t u[4];
+                u8_of<2>(w[i], u);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) o[8 * q + 4 * i + j] = s8_of<2>(u[j]);
+            }
+        } else {
+            uint4 x, y;
+            if (P >= 32) {
+                x = *reinterpret_cast<const uint4*>(row + in);
+                y = *reinterpret_cast<const uint4*>(row + in + 16);
+            } else {
+                x = *reinterpret_cast<const uint4*>(row);
+                y = *reinterpret_cast<const uint4*>(row + bb);
+            }
+            o[8 * q + 0] = s8_of<8>(x.x); o[8 * q + 1] = s8_of<8>(x.y);
+            o[8 * q + 2] = s8_of<8>(x.z); o[8 * q + 3] = s8_of<8>(x.w);
+            o[8 * q + 4] = s8_of<8>(y.x); o[8 * q + 5] = s8_of<8>(y.y);
+            o[8 * q + 6] = s8_of<8>(y.z); o[8 * q + 7] = s8_of<8>(y.w);
+        }
+    }
+}
+
+__device__ __forceinline__ void umma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}"
+                 :: "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+
+// balanced signed byte digits of x (|x| < 2^22): x = d0 + 256 d1 + 65536 d2
+__device__ __forceinline__ void digits3(int x, int& d0, int& d1, int& d2)
+{
+    d0 = (int)(int8_t)(x & 0xFF);
+    const int r1 = (x - d0) >> 8;
+    d1 = (int)(int8_t)(r1 & 0xFF);
+    d2 = (r1 - d1) >> 8;
+}
+
+template <int BITS, int RG>
+__global__ void __launch_bounds__(kTcThreads, 4)
+k_decode_i8(const TcArgs a)
+{
+    using F = I8Fmt<BITS>;
+    constexpr int NS = 4 * RG;                       // S / O columns: 4r + digit
+    constexpr uint32_t kColAK = 0, kColAV = 32, kColS = 64, kColO = 64 + NS;
+    // kind::i8, s32 accumulate, M = 128, N = NS.  S: A u8, B s8 K-major.
+    // O: A s8, B u8 MN-major.
+    constexpr uint32_t kIdescS = (2u << 4) | (0u << 7) | (1u << 10) |
+                                 ((uint32_t)(NS >> 3) << 17) | (8u << 24);
+    constexpr uint32_t kIdescO = (2u << 4) | (1u << 7) | (0u << 10) | (1u << 16) |
+                                 ((uint32_t)(NS >> 3) << 17) | (8u << 24);
+    constexpr uint32_t kQRow = (NS / 8) * 128;      // bytes per 16-deep K chunk of q''
+    constexpr uint32_t kPRow = (NS / 16) * 128;     // bytes per 8-deep K group of P''
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* bar_s = full + kStages;
+    uint64_t* bar_o = bar_s + 1;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + 64);
+    int* s_flag = reinterpret_cast<int*>(smem + 68);
+    float* s_red = reinterpret_cast<float*>(smem + 128);             // [4][16]
+    unsigned* s_redv = reinterpret_cast<unsigned*>(smem + 384);      // [4]
+    float* s_rowfac = reinterpret_cast<float*>(smem + 400);          // [16]
+    float* s_l = reinterpret_cast<float*>(smem + 464);               // [4][16]
+    int* s_init = reinterpret_cast<int*>(smem + 768);                // [NS] accumulator start
+    uint8_t* s_qb = smem + 1024;                                     // q'' digits: 128 x NS bytes
+    uint8_t* s_pb = s_qb + 128 * NS;                                 // P'' digits: 128 x NS bytes
+    float* s_qf = reinterpret_cast<float*>(s_pb + 128 * NS);         // [RG][128] staging
+    uint8_t* ring = reinterpret_cast<uint8_t*>(s_qf) + RG * 512;
+
+    const int split = blockIdx.x;
+    const int b = blockIdx.z;
+    const int kvh = blockIdx.y / a.R;
+    const int rg = blockIdx.y - kvh * a.R;
+    const int seq_len = a.seq_lens[b];
+    if (seq_len < a.q_len || seq_len > a.max_seq_len) {
+        if (split == 0 && blockIdx.y == 0 && threadIdx.x == 0)
+            report_error(a.err, TQ_ERR_DEVICE_CHECK, kErrSeqLen);
+        return;
+    }
+    const int nsplit = (seq_len + a.split_tokens - 1) / a.split_tokens;
+    if (split >= nsplit) return;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tok_begin = split * a.split_tokens;
+    const int tok_end = min(seq_len, tok_begin + a.split_tokens);
+    const int ntiles = (tok_end - tok_begin + kTile - 1) / kTile;
+    const int P = a.page_size;
+    const int npp = kTile / P;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+        mbar_init(bar_s, 1);
+        mbar_init(bar_o, 1);
+        s_flag[0] = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(s_tmem, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    const uint32_t t_lane = tmem + ((uint32_t)(32 * warp) << 16);
+
+    if (warp == 0) {
+        for (int s = 0; s < kStages && s < ntiles; ++s) {
+            const int t0 = tok_begin + s * kTile;
+            issue_tile_tc(ring + s * F::kStage, &full[s], a, b, kvh, t0, min(kTile, tok_end - t0),
+                          lane);
+        }
+    }
+
+    // ---- query rows: rotate, log2 scale, fixed point q'' with |q''| < 2^22
+    for (int rr = warp; rr < RG; rr += 4) {
+        const int r = rg * RG + rr;
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        if (r < a.G) {
+            const int tq = r / a.group;
+            const int h = kvh * a.group + (r - tq * a.group);
+            const uint2 raw = __ldg(reinterpret_cast<const uint2*>(
+                a.q + (((int64_t)b * a.q_len + tq) * a.num_q_heads + h) * kHeadDim) + lane);
+            x[0] = bf16_bits_to_float(raw.x & 0xffffu);
+            x[1] = bf16_bits_to_float(raw.x >> 16);
+            x[2] = bf16_bits_to_float(raw.y & 0xffffu);
+            x[3] = bf16_bits_to_float(raw.y >> 16);
+        }
+        fwht128_lane(x, lane);
+        float amax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            x[e] *= kLog2eTc / kHeadDim;
+            amax = fmaxf(amax, fabsf(x[e]));
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, m));
+        const int ex = amax > 0.f ? max(-100, ilogbf(amax)) : 0;
+        const float pre = pow2i(21 - ex);           // largest |q''| in [2^21, 2^22)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s_qf[rr * kHeadDim + 4 * lane + e] = rintf(x[e] * pre);
+        if (lane == 0) s_rowfac[rr] = pow2i(ex - 21);
+    }
+    __syncthreads();
+    {
+        // K position k = tid holds dimension perm(k); column 4r + d holds
+        // digit d of row r (d = 3: zero)
+        const int k = tid;
+        const int dim = perm_i8<BITS>(k);
+        int dsum[3 * RG];
+#pragma unroll
+        for (int r = 0; r < RG; ++r) {
+            int d0, d1, d2;
+            digits3((int)s_qf[r * kHeadDim + dim], d0, d1, d2);
+            const int dd[4] = {d0, d1, d2, 0};
+#pragma unroll
+            for (int d = 0; d < 4; ++d) {
+                const int n = 4 * r + d;
+                const int cm = (k >> 4) * (NS / 8) + (n >> 3);
+                s_qb[cm * 128 + (n & 7) * 16 + (k & 15)] = (uint8_t)(int8_t)dd[d];
+                if (d < 3) dsum[3 * r + d] = dd[d];
+            }
+        }
+        // accumulator start: -L * (sum over dims of each digit column), summed
+        // per warp by shuffles, then over the 4 warps in the (idle) P'' buffer
+#pragma unroll
+        for (int i = 0; i < 3 * RG; ++i) {
+            int v = dsum[i];
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
+            dsum[i] = v;
+        }
+        int* s_sum = reinterpret_cast<int*>(s_pb);                   // [4][3 RG]
+        if (lane == 0)
+#pragma unroll
+            for (int i = 0; i < 3 * RG; ++i) s_sum[warp * 3 * RG + i] = dsum[i];
+        __syncthreads();
+        if (tid < NS) {
+            const int r = tid >> 2, d = tid & 3;
+            int v = 0;
+            if (d < 3)
+                for (int w = 0; w < 4; ++w) v += s_sum[w * 3 * RG + 3 * r + d];
+            s_init[tid] = -F::L * v;
+        }
+    }
+    float rowfac[RG];
+    int lim[RG];
+#pragma unroll
+    for (int r = 0; r < RG; ++r) {
+        rowfac[r] = s_rowfac[r];
+        const int R = rg * RG + r;
+        lim[r] = R < a.G ? seq_len - a.q_len + R / a.group : -1;
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    uint32_t sinit[NS];
+#pragma unroll
+    for (int n = 0; n < NS; ++n) sinit[n] = (uint32_t)s_init[n];
+    const uint64_t desc_q = smem_desc(s_qb, kQRow, 128);
+    const uint64_t desc_p = smem_desc(s_pb, kPRow, 128);
+
+    float m_run[RG], l_run[RG], o_reg[RG];
+#pragma unroll
+    for (int r = 0; r < RG; ++r) {
+        m_run[r] = -CUDART_INF_F;
+        l_run[r] = 0.f;
+        o_reg[r] = 0.f;
+    }
+    int ev = 0;
+    float vn = 1.f;
+    float vlimit = __uint_as_float(1u << 23);
+    const float kinv = 1.f / (float)F::L;
+    const int lim_min = seq_len - a.q_len + (rg * RG) / a.group;
+    const int kpos = perm_i8_inv<BITS>(tid);
+    bool aborted = false;
+    bool o_acc = false;                 // O holds an int32 sum to extend
+
+    // fold O (int32 digit sums, scale 2^(ev - 127) 2^-22) into o_reg (dimension tid)
+    auto flush_o = [&](float scale_now) {
+        uint32_t ov[NS];
+#pragma unroll
+        for (int c = 0; c < NS; c += 16) tmem_ld16(t_lane + kColO + c, ov + c);
+        tmem_wait_ld();
+#pragma unroll
+        for (int r = 0; r < RG; ++r) {
+            float v = (float)(int)ov[4 * r + 3];
+            v = fmaf(v, 256.f, (float)(int)ov[4 * r + 2]);
+            v = fmaf(v, 256.f, (float)(int)ov[4 * r + 1]);
+            v = fmaf(v, 256.f, (float)(int)ov[4 * r]);
+            o_reg[r] = fmaf(v, scale_now, o_reg[r]);
+        }
+    };
+
+    for (int tt = 0; tt < ntiles; ++tt) {
+        const int stage = tt % kStages;
+        uint8_t* st = ring + stage * F::kStage;
+        const int tok0 = tok_begin + tt * kTile;
+        bool ok = mbar_wait_sleep(&full[stage], (uint32_t)((tt / kStages) & 1), kPollsTc);
+        tc_fence_after();
+        if (!ok) atomicOr(&s_flag[0], 1);
+
+        // K row of token tid -> A (u8); accumulator start -> S
+        const int pg = tid / P, row = tid % P;
+        const uint8_t* kblk = st + pg * a.block_bytes;
+        const uint8_t* vblk = st + (npp + pg) * a.block_bytes;
+        k_row_to_tmem_u8<BITS>(kblk + row * F::CB, t_lane + kColAK);
+#pragma unroll
+        for (int c = 0; c < NS; c += 16) tmem_st16(t_lane + kColS + c, sinit + c);
+        float ks = reinterpret_cast<const float*>(kblk + P * F::CB)[row] * kinv;
+        float vs = reinterpret_cast<const float*>(vblk + P * F::CB)[row] * kinv;
+        const int tok = tok0 + tid;
+        if (tok >= tok_end) { ks = 0.f; vs = 0.f; }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+        if (s_flag[0]) { aborted = true; break; }
+
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                umma_i8_ts(tmem + kColS, tmem + kColAK + 8 * j, desc_q + ((2 * j * kQRow) >> 4),
+                           kIdescS, 1u);
+            umma_commit(bar_s);
+        }
+
+        // V column of dimension tid (registers) while S is computed
+        uint32_t vw[32];
+        v_col_s8<BITS>(st + npp * a.block_bytes, a.block_bytes, P, tid, vw);
+        if (tt > 0) {
+            ok = mbar_wait_sleep(bar_o, (uint32_t)((tt - 1) & 1), kPollsTc);
+            tc_fence_after();
+            if (!ok) atomicOr(&s_flag[0], 1);
+        }
+        tmem_st16(t_lane + kColAV, vw);
+        tmem_st16(t_lane + kColAV + 16, vw + 16);
+
+        ok = mbar_wait_sleep(bar_s, (uint32_t)(tt & 1), kPollsTc);
+        tc_fence_after();
+        if (!ok) atomicOr(&s_flag[0], 1);
+        uint32_t sraw[NS];
+#pragma unroll
+        for (int c = 0; c < NS; c += 16) tmem_ld16(t_lane + kColS + c, sraw + c);
+        tmem_wait_ld();
+
+        const bool full_tile = tok0 + kTile - 1 <= lim_min;
+        float sc[RG];
+        bool need = false;
+#pragma unroll
+        for (int r = 0; r < RG; ++r) {
+            float v = fmaf((float)(int)sraw[4 * r + 2], 65536.f, (float)(int)sraw[4 * r + 1] * 256.f);
+            v += (float)(int)sraw[4 * r];
+            float x = v * (ks * rowfac[r]);
+            if (!full_tile) x = tok <= lim[r] ? x : -CUDART_INF_F;
+            sc[r] = x;
+            need |= x > m_run[r] + kLazyTc;
+        }
+        need |= vs >= vlimit;
+        const int any = __syncthreads_or(need);
+        if (s_flag[0]) { aborted = true; break; }
+        if (warp == 0 && tt + kStages < ntiles) {
+            const int t0 = tok_begin + (tt + kStages) * kTile;
+            issue_tile_tc(st, &full[stage], a, b, kvh, t0, min(kTile, tok_end - t0), lane);
+        }
+        if (any) {
+#pragma unroll
+            for (int r = 0; r < RG; ++r) {
+                float v = sc[r];
+#pragma unroll
+                for (int m = 16; m >= 1; m >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, m));
+                if (lane == 0) s_red[warp * 16 + r] = v;
+            }
+            const unsigned vb = __reduce_max_sync(kFull, __float_as_uint(vs));
+            if (lane == 0) s_redv[warp] = vb;
+            __syncthreads();
+            // fold the running int32 O (old scale) into o_reg, then rescale
+            if (o_acc) flush_o(pow2i(ev - 127 - 22));
+            o_acc = false;
+            const unsigned vmax = max(max(s_redv[0], s_redv[1]), max(s_redv[2], s_redv[3]));
+            ev = max(ev, (int)(vmax >> 23));
+            vn = pow2i(127 - ev);
+            vlimit = ev >= 254 ? CUDART_INF_F : __uint_as_float((uint32_t)(ev + 1) << 23);
+#pragma unroll
+            for (int r = 0; r < RG; ++r) {
+                const float tmax = fmaxf(fmaxf(s_red[r], s_red[16 + r]),
+                                         fmaxf(s_red[32 + r], s_red[48 + r]));
+                const float mn = fmaxf(m_run[r], tmax);
+                const float alpha = mn == -CUDART_INF_F ? 1.f : fast_exp2(m_run[r] - mn);
+                m_run[r] = mn;
+                l_run[r] *= alpha;
+                o_reg[r] *= alpha;
+            }
+            __syncthreads();
+        }
+
+        // P'' row of token tid at K position kpos: 4 digit bytes per row
+        const float vn_t = vs * vn * 4194304.f;       // 2^22 fixed point
+        uint32_t pw[RG];
+#pragma unroll
+        for (int r = 0; r < RG; ++r) {
+            float pr = fast_exp2(sc[r] - m_run[r]);
+            if (!full_tile) pr = sc[r] == -CUDART_INF_F ? 0.f : pr;
+            l_run[r] += pr;
+            pw[r] = pr > 0.f ? __float2uint_rn(pr * vn_t) : 0u;
+        }
+        {
+            uint8_t* rowp = s_pb + (kpos >> 3) * kPRow + (kpos & 7) * 16;
+#pragma unroll
+            for (int ng = 0; ng < RG / 4; ++ng)
+                *reinterpret_cast<uint4*>(rowp + ng * 128) =
+                    make_uint4(pw[4 * ng], pw[4 * ng + 1], pw[4 * ng + 2], pw[4 * ng + 3]);
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                umma_i8_ts(tmem + kColO, tmem + kColAV + 8 * j, desc_p + ((4 * j * kPRow) >> 4),
+                           kIdescO, (o_acc || j > 0) ? 1u : 0u);
+            umma_commit(bar_o);
+        }
+        o_acc = true;
+    }
+
+    // ---- epilogue
+    bool ok = !aborted && mbar_wait_sleep(bar_o, (uint32_t)((ntiles - 1) & 1), kPollsTc);
+    tc_fence_after();
+    const int nrows = min(RG, a.G - rg * RG);
+    float* sO = reinterpret_cast<float*>(ring);          // [RG][128]
+    if (ok) {
+        if (o_acc) flush_o(pow2i(ev - 127 - 22));
+#pragma unroll
+        for (int r = 0; r < RG; ++r) sO[r * kHeadDim + tid] = o_reg[r];
+#pragma unroll
+        for (int r = 0; r < RG; ++r) {
+            float l = l_run[r];
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) l += __shfl_xor_sync(kFull, l, m);
+            if (lane == 0) s_l[warp * 16 + r] = l;
+        }
+    } else if (tid == 0) {
+        report_error(a.err, TQ_ERR_TIMEOUT, kErrWaitTile);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+    if (!ok) return;
+    tc_finish<RG>(a, sO, s_l, m_run, s_flag, b, kvh, rg, split, nsplit, nrows, warp, lane, tid);
+}
+
+template <int BITS, int RG>
 cudaError_t launch_tc(const TcArgs& a, dim3 grid, cudaStream_t stream)
 {
+    constexpr int NCOL = 2 * RG < 16 ? 16 : 2 * RG;
     const size_t smem = 1024 + 2 * 256 * NCOL + (size_t)kStages * TcFmt<BITS>::kStage;
     static int configured = 0;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 31 || !(configured & (1 << dev))) {
-        e = cudaFuncSetAttribute(k_decode_tc<BITS, NCOL>,
+        e = cudaFuncSetAttribute(k_decode_tc<BITS, RG>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         if (dev < 31) configured |= 1 << dev;
     }
-    k_decode_tc<BITS, NCOL><<<grid, kTcThreads, smem, stream>>>(a);
+    k_decode_tc<BITS, RG><<<grid, kTcThreads, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+template <int BITS, int RG>
+cudaError_t launch_i8(const TcArgs& a, dim3 grid, cudaStream_t stream)
+{
+    constexpr int NS = 4 * RG;
+    const size_t smem = 1024 + 2 * 128 * NS + RG * 512 + (size_t)kStages * I8Fmt<BITS>::kStage;
+    static int configured = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 31 || !(configured & (1 << dev))) {
+        e = cudaFuncSetAttribute(k_decode_i8<BITS, RG>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        if (dev < 31) configured |= 1 << dev;
+    }
+    k_decode_i8<BITS, RG><<<grid, kTcThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-// rows of one tensor-core CTA: 8 (N = 16) when G <= 8, else 16 (N = 32)
-int decode_tc_rows(int G) { return G <= 8 ? 8 : 16; }
+// Query rows of one tensor-core CTA.  The integer kernel (2-, 4- and 8-bit
+// codes) takes 4 or 8; the f16 kernel (3-bit codes) 4, 8 or 16.
+int decode_tc_rows(int format, int G)
+{
+    if (format == 3) return G <= 4 ? 4 : (G <= 8 ? 8 : 16);
+    return G <= 4 ? 4 : 8;
+}
 
 cudaError_t launch_decode_tc(const void* q, const tq_cache& c, int64_t block_bytes,
                              const int32_t* page_table, int max_pages, const int32_t* seq_lens,
@@ -721,7 +1311,7 @@ cudaError_t launch_decode_tc(const void* q, const tq_cache& c, int64_t block_byt
     a.group = num_q_heads / c.num_kv_heads;
     a.q_len = q_len;
     a.G = q_len * a.group;
-    const int rows = decode_tc_rows(a.G);
+    const int rows = decode_tc_rows(c.format, a.G);
     a.R = (a.G + rows - 1) / rows;
     a.page_size = c.page_size;
     a.split_tokens = split_tokens;
@@ -737,16 +1327,18 @@ cudaError_t launch_decode_tc(const void* q, const tq_cache& c, int64_t block_byt
         a.ws_o = reinterpret_cast<float*>(w + cnt + ml);
     }
     const dim3 grid((unsigned)a.max_splits, (unsigned)(c.num_kv_heads * a.R), (unsigned)batch);
-#define TQ_TC(B) \
-    return rows == 8 ? launch_tc<B, 16>(a, grid, stream) : launch_tc<B, 32>(a, grid, stream)
+#define TQ_I8(B) return rows == 4 ? launch_i8<B, 4>(a, grid, stream) : launch_i8<B, 8>(a, grid, stream)
     switch (c.format) {
-    case 2: TQ_TC(2);
-    case 3: TQ_TC(3);
-    case 4: TQ_TC(4);
-    case 8: TQ_TC(8);
+    case 2: TQ_I8(2);
+    case 3:
+        return rows == 4   ? launch_tc<3, 4>(a, grid, stream)
+               : rows == 8 ? launch_tc<3, 8>(a, grid, stream)
+                           : launch_tc<3, 16>(a, grid, stream);
+    case 4: TQ_I8(4);
+    case 8: TQ_I8(8);
     default: return cudaErrorInvalidValue;
     }
-#undef TQ_TC
+#undef TQ_I8
 }
 
 }  // namespace tq

@@ -65,12 +65,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     return ok != 0;
 }
 
+// try_wait that may suspend the thread for up to `ns` nanoseconds while the
+// phase is incomplete (no busy polling).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity), "r"(ns) : "memory");
+    return ok != 0;
+}
+
 // Bounded wait: false when the phase did not complete within `spins` polls.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   uint32_t spins)
 {
     for (uint32_t i = 0; i < spins; ++i)
         if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+// Bounded sleeping wait: each poll suspends up to 20 us, at most `polls`
+// polls (the whole wait is bounded by polls x 20 us).
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t polls)
+{
+    for (uint32_t i = 0; i < polls; ++i)
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     return false;
 }
 

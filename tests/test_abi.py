@@ -113,16 +113,43 @@ def test_decode_validation():
     assert dec(c, max_len=4, q_len=8) == I            # max_seq_len < q_len
 
 
+def _expected_workspace(batch, Hkv, G, seq, P, fmt):
+    """Workspace layout the decode kernels use: merge counters, then (m, l)
+    and the 128-float partial output of every (unit, split, row), where a
+    unit is one (sequence, kv head, row group).  Rows per CTA: 8 for the bf16
+    cache; 4 or 8 for turbo2/4/8; 4, 8 or 16 for turbo3.  Splits are 2048
+    tokens (1024 with 64-token pages)."""
+    split = 1024 if P == 64 else 2048
+    nsplit = -(-seq // split)
+    if nsplit <= 1:
+        return 0
+    if fmt == 16:
+        rows = 8
+    elif fmt == 3:
+        rows = 4 if G <= 4 else (8 if G <= 8 else 16)
+    else:
+        rows = 4 if G <= 4 else 8
+    units = batch * Hkv * -(-G // rows)
+    r256 = lambda x: -(-x // 256) * 256
+    return r256(units * 4) + r256(units * nsplit * rows * 8) + units * nsplit * rows * 128 * 4
+
+
 def test_workspace_size():
-    c = desc()
     ws = tq.lib().tq_decode_workspace_size
+    c = desc()
     # one split (<= 2048 tokens with 16-token pages): no workspace
     assert ws(8, 1, 32, 2048, ctypes.byref(c)) == 0
-    n = ws(8, 1, 32, 8192, ctypes.byref(c))
-    # 4 splits x 64 (seq, kv head) units x 8 rows x (128 + 2) floats + counters
-    assert n >= 4 * 64 * 8 * 130 * 4 and n < 4 * 64 * 8 * 130 * 4 + 4096
+    assert ws(8, 1, 32, 2049, ctypes.byref(c)) == _expected_workspace(8, 8, 4, 2049, 16, 4)
+    # 4 splits x 64 (seq, kv head) units x 4 rows x (128 + 2) floats + counters
+    assert ws(8, 1, 32, 8192, ctypes.byref(c)) == 4 * 64 * 4 * 130 * 4 + 256
     assert ws(8, 1, 30, 4096, ctypes.byref(c)) == 0   # invalid
+    for fmt in (2, 3, 4, 8, 16):
+        for q_len, Hq in ((1, 32), (1, 64), (4, 32), (8, 64), (3, 40)):
+            cf = desc(fmt=fmt)
+            assert ws(8, q_len, Hq, 8192, ctypes.byref(cf)) == \
+                _expected_workspace(8, 8, q_len * Hq // 8, 8192, 16, fmt), (fmt, q_len, Hq)
     c64 = desc(P=64)
+    assert ws(4, 1, 40, 131072, ctypes.byref(c64)) == _expected_workspace(4, 8, 5, 131072, 64, 4)
     assert ws(4, 1, 40, 131072, ctypes.byref(c64)) >= 4 * 8 * 128 * 8 * 130 * 4
 
 
