@@ -65,6 +65,7 @@ struct TcArgs {
     int G;
     int R;             // row groups
     int page_size;
+    int lp;            // log2(page_size)
     int split_tokens;
     int max_splits;
     int max_seq_len;
@@ -194,17 +195,18 @@ __device__ __forceinline__ void k_row_to_tmem(const uint8_t* row, uint32_t taddr
 // columns [0, 64) of this thread's lane.  vblk0: first V block of the tile in
 // the stage; pages of P tokens follow each other every block_bytes.
 template <int BITS>
-__device__ __forceinline__ void v_col_to_tmem(const uint8_t* vblk0, int64_t bb, int P, int dim,
+__device__ __forceinline__ void v_col_to_tmem(const uint8_t* vblk0, int64_t bb, int lp, int dim,
                                               uint32_t taddr)
 {
+    const int P = 1 << lp;
     uint32_t o[16];
     // tokens are emitted 16 pairs (32 tokens) per store
     const int row_bytes = P * BITS / 8;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const int t0 = 32 * q;                   // first tile token of this chunk
-        const int pg = t0 / P;                   // page holding it
-        const int in = t0 % P;                   // its offset in the page
+        const int pg = t0 >> lp;                 // page holding it
+        const int in = t0 & (P - 1);             // its offset in the page
         const uint8_t* row = vblk0 + pg * bb + (int64_t)dim * row_bytes;
         if constexpr (BITS == 4) {
             // 32 tokens = 16 bytes of one row (P >= 32) or two 8-byte rows (P = 16)
@@ -263,16 +265,17 @@ __device__ __forceinline__ void v_col_to_tmem(const uint8_t* vblk0, int64_t bb, 
 }
 
 // Bulk copies of one tile's K and V page blocks into a stage (warp 0).
+// pids[j]: physical page of the tile's j-th page (global page table or the
+// split's copy in shared memory).
 __device__ __forceinline__ void issue_tile_tc(uint8_t* stage, uint64_t* bar, const TcArgs& a,
-                                              int b, int kvh, int tok0, int ntok, int lane)
+                                              const int* pids, int kvh, int ntok, int lane)
 {
-    const int P = a.page_size;
-    const int npp = kTile / P;                          // page slots per stage
-    const int npg = (ntok + P - 1) / P;                 // pages holding tokens
+    const int npp = kTile >> a.lp;                        // page slots per stage
+    const int npg = (ntok + (1 << a.lp) - 1) >> a.lp;     // pages holding tokens
     if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(2 * npg * a.block_bytes));
     __syncwarp();
     if (lane < npg) {
-        int pid = __ldg(a.page_table + (int64_t)b * a.max_pages + tok0 / P + lane);
+        int pid = pids[lane];
         if (pid < 0 || pid >= a.num_pages) {
             report_error(a.err, TQ_ERR_DEVICE_CHECK, kErrPageRange);
             pid = 0;
@@ -281,6 +284,15 @@ __device__ __forceinline__ void issue_tile_tc(uint8_t* stage, uint64_t* bar, con
         bulk_g2s(stage + lane * a.block_bytes, a.kp + off, (uint32_t)a.block_bytes, bar);
         bulk_g2s(stage + (npp + lane) * a.block_bytes, a.vp + off, (uint32_t)a.block_bytes, bar);
     }
+}
+
+// The split's page ids -> shared memory (at most 128: 2048 tokens of 16).
+__device__ __forceinline__ void load_split_pids(int* s_pid, const TcArgs& a, int b, int tok_begin,
+                                                int tok_end, int tid)
+{
+    const int first = tok_begin >> a.lp;
+    const int n = ((tok_end - 1) >> a.lp) - first + 1;
+    if (tid < n) s_pid[tid] = __ldg(a.page_table + (int64_t)b * a.max_pages + first + tid);
 }
 
 // Split epilogue shared by the tensor-core kernels.  sO: the split's
@@ -386,7 +398,8 @@ k_decode_tc(const TcArgs a)
     unsigned* s_redv = reinterpret_cast<unsigned*>(smem + 384);      // [4]
     float* s_rowfac = reinterpret_cast<float*>(smem + 400);          // [16]
     float* s_l = reinterpret_cast<float*>(smem + 464);               // [4][16]
-    uint8_t* s_qb = smem + 1024;                                     // Q' operand
+    int* s_pid = reinterpret_cast<int*>(smem + 1024);                // [128] split page ids
+    uint8_t* s_qb = smem + 1536;                                     // Q' operand
     uint8_t* s_pb = s_qb + 256 * NCOL;                               // P' operand / q staging
     uint8_t* ring = s_pb + 256 * NCOL;
 
@@ -408,7 +421,7 @@ k_decode_tc(const TcArgs a)
     const int tok_end = min(seq_len, tok_begin + a.split_tokens);
     const int ntiles = (tok_end - tok_begin + kTile - 1) / kTile;
     const int P = a.page_size;
-    const int npp = kTile / P;
+    const int npp = kTile >> a.lp;
 
     // ---- set-up: barriers, tensor memory, first copies
     if (tid == 0) {
@@ -431,10 +444,13 @@ k_decode_tc(const TcArgs a)
     if (warp == 0) {
         for (int s = 0; s < kStages && s < ntiles; ++s) {
             const int t0 = tok_begin + s * kTile;
-            issue_tile_tc(ring + s * F::kStage, &full[s], a, b, kvh, t0, min(kTile, tok_end - t0),
-                          lane);
+            issue_tile_tc(ring + s * F::kStage, &full[s], a,
+                          a.page_table + (int64_t)b * a.max_pages + (t0 >> a.lp), kvh,
+                          min(kTile, tok_end - t0), lane);
         }
     }
+
+    load_split_pids(s_pid, a, b, tok_begin, tok_end, tid);   // visible after the next barrier
 
     // ---- query rows of this row group: rotate, scale to log2 units,
     // power-of-two prescale (hi and lo parts stay normal f16)
@@ -528,7 +544,7 @@ k_decode_tc(const TcArgs a)
         if (!ok) atomicOr(&s_flag[0], 1);
 
         // 1. K row of token tid -> A operand
-        const int pg = tid / P, row = tid % P;
+        const int pg = tid >> a.lp, row = tid & (P - 1);
         const uint8_t* kblk = st + pg * a.block_bytes;
         const uint8_t* vblk = st + (npp + pg) * a.block_bytes;
         k_row_to_tmem<BITS>(kblk + row * F::CB, t_lane);
@@ -558,7 +574,7 @@ k_decode_tc(const TcArgs a)
         uint32_t sraw[NCOL];
 #pragma unroll
         for (int c = 0; c < NCOL; c += 16) tmem_ld16(t_lane + kColS + c, sraw + c);
-        v_col_to_tmem<BITS>(st + npp * a.block_bytes, a.block_bytes, P, tid, t_lane);
+        v_col_to_tmem<BITS>(st + npp * a.block_bytes, a.block_bytes, a.lp, tid, t_lane);
         tmem_wait_ld();
         const bool full_tile = tok0 + kTile - 1 <= lim_min;
         float sc[RG];
@@ -575,7 +591,8 @@ k_decode_tc(const TcArgs a)
         if (s_flag[0]) { aborted = true; break; }
         if (warp == 0 && tt + kStages < ntiles) {
             const int t0 = tok_begin + (tt + kStages) * kTile;
-            issue_tile_tc(st, &full[stage], a, b, kvh, t0, min(kTile, tok_end - t0), lane);
+            issue_tile_tc(st, &full[stage], a, s_pid + ((t0 - tok_begin) >> a.lp), kvh,
+                          min(kTile, tok_end - t0), lane);
         }
         if (any) {
             // exact tile maxima of every row and of the V scales
@@ -805,15 +822,16 @@ __device__ __forceinline__ void k_row_to_tmem_u8(const uint8_t* row, uint32_t ta
 // signed bytes in K-position order (registers; stored once the previous
 // PV product has drained).
 template <int BITS>
-__device__ __forceinline__ void v_col_s8(const uint8_t* vblk0, int64_t bb, int P, int dim,
+__device__ __forceinline__ void v_col_s8(const uint8_t* vblk0, int64_t bb, int lp, int dim,
                                          uint32_t* o)
 {
+    const int P = 1 << lp;
     // 32 tokens per chunk: 16 bytes (4-bit), 8 bytes (2-bit), 32 bytes (8-bit)
     const int row_bytes = P * BITS / 8;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const int t0 = 32 * q;
-        const int pg = t0 / P, in = t0 % P;
+        const int pg = t0 >> lp, in = t0 & (P - 1);
         const uint8_t* row = vblk0 + pg * bb + (int64_t)dim * row_bytes;
         uint32_t w[8];
         if constexpr (BITS == 4) {
@@ -910,7 +928,8 @@ k_decode_i8(const TcArgs a)
     float* s_rowfac = reinterpret_cast<float*>(smem + 400);          // [16]
     float* s_l = reinterpret_cast<float*>(smem + 464);               // [4][16]
     int* s_init = reinterpret_cast<int*>(smem + 768);                // [NS] accumulator start
-    uint8_t* s_qb = smem + 1024;                                     // q'' digits: 128 x NS bytes
+    int* s_pid = reinterpret_cast<int*>(smem + 1024);                // [128] split page ids
+    uint8_t* s_qb = smem + 1536;                                     // q'' digits: 128 x NS bytes
     uint8_t* s_pb = s_qb + 128 * NS;                                 // P'' digits: 128 x NS bytes
     float* s_qf = reinterpret_cast<float*>(s_pb + 128 * NS);         // [RG][128] staging
     uint8_t* ring = reinterpret_cast<uint8_t*>(s_qf) + RG * 512;
@@ -933,7 +952,7 @@ k_decode_i8(const TcArgs a)
     const int tok_end = min(seq_len, tok_begin + a.split_tokens);
     const int ntiles = (tok_end - tok_begin + kTile - 1) / kTile;
     const int P = a.page_size;
-    const int npp = kTile / P;
+    const int npp = kTile >> a.lp;
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
@@ -955,10 +974,13 @@ k_decode_i8(const TcArgs a)
     if (warp == 0) {
         for (int s = 0; s < kStages && s < ntiles; ++s) {
             const int t0 = tok_begin + s * kTile;
-            issue_tile_tc(ring + s * F::kStage, &full[s], a, b, kvh, t0, min(kTile, tok_end - t0),
-                          lane);
+            issue_tile_tc(ring + s * F::kStage, &full[s], a,
+                          a.page_table + (int64_t)b * a.max_pages + (t0 >> a.lp), kvh,
+                          min(kTile, tok_end - t0), lane);
         }
     }
+
+    load_split_pids(s_pid, a, b, tok_begin, tok_end, tid);   // visible after the next barrier
 
     // ---- query rows: rotate, log2 scale, fixed point q'' with |q''| < 2^22
     for (int rr = warp; rr < RG; rr += 4) {
@@ -1088,7 +1110,7 @@ k_decode_i8(const TcArgs a)
         if (!ok) atomicOr(&s_flag[0], 1);
 
         // K row of token tid -> A (u8); accumulator start -> S
-        const int pg = tid / P, row = tid % P;
+        const int pg = tid >> a.lp, row = tid & (P - 1);
         const uint8_t* kblk = st + pg * a.block_bytes;
         const uint8_t* vblk = st + (npp + pg) * a.block_bytes;
         k_row_to_tmem_u8<BITS>(kblk + row * F::CB, t_lane + kColAK);
@@ -1114,7 +1136,7 @@ k_decode_i8(const TcArgs a)
 
         // V column of dimension tid (registers) while S is computed
         uint32_t vw[32];
-        v_col_s8<BITS>(st + npp * a.block_bytes, a.block_bytes, P, tid, vw);
+        v_col_s8<BITS>(st + npp * a.block_bytes, a.block_bytes, a.lp, tid, vw);
         if (tt > 0) {
             ok = mbar_wait_sleep(bar_o, (uint32_t)((tt - 1) & 1), kPollsTc);
             tc_fence_after();
@@ -1148,7 +1170,8 @@ k_decode_i8(const TcArgs a)
         if (s_flag[0]) { aborted = true; break; }
         if (warp == 0 && tt + kStages < ntiles) {
             const int t0 = tok_begin + (tt + kStages) * kTile;
-            issue_tile_tc(st, &full[stage], a, b, kvh, t0, min(kTile, tok_end - t0), lane);
+            issue_tile_tc(st, &full[stage], a, s_pid + ((t0 - tok_begin) >> a.lp), kvh,
+                          min(kTile, tok_end - t0), lane);
         }
         if (any) {
 #pragma unroll
@@ -1246,7 +1269,7 @@ template <int BITS, int RG>
 cudaError_t launch_tc(const TcArgs& a, dim3 grid, cudaStream_t stream)
 {
     constexpr int NCOL = 2 * RG < 16 ? 16 : 2 * RG;
-    const size_t smem = 1024 + 2 * 256 * NCOL + (size_t)kStages * TcFmt<BITS>::kStage;
+    const size_t smem = 1536 + 2 * 256 * NCOL + (size_t)kStages * TcFmt<BITS>::kStage;
     static int configured = 0;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1265,7 +1288,7 @@ template <int BITS, int RG>
 cudaError_t launch_i8(const TcArgs& a, dim3 grid, cudaStream_t stream)
 {
     constexpr int NS = 4 * RG;
-    const size_t smem = 1024 + 2 * 128 * NS + RG * 512 + (size_t)kStages * I8Fmt<BITS>::kStage;
+    const size_t smem = 1536 + 2 * 128 * NS + RG * 512 + (size_t)kStages * I8Fmt<BITS>::kStage;
     static int configured = 0;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1314,6 +1337,7 @@ cudaError_t launch_decode_tc(const void* q, const tq_cache& c, int64_t block_byt
     const int rows = decode_tc_rows(c.format, a.G);
     a.R = (a.G + rows - 1) / rows;
     a.page_size = c.page_size;
+    a.lp = c.page_size == 16 ? 4 : (c.page_size == 32 ? 5 : 6);
     a.split_tokens = split_tokens;
     a.max_splits = (max_seq_len + split_tokens - 1) / split_tokens;
     a.max_seq_len = max_seq_len;
