@@ -286,6 +286,31 @@ __device__ __forceinline__ void issue_tile_tc(uint8_t* stage, uint64_t* bar, con
     }
 }
 
+// The same copies spread over the CTA's 4 warps: warp w takes pages
+// w, w + 4, ...; each warp's lane 0 arrives with its own byte count (the
+// stage barrier counts 4 arrivals), so no warp waits on another to issue.
+__device__ __forceinline__ void issue_tile_warps(uint8_t* stage, uint64_t* bar, const TcArgs& a,
+                                                 const int* pids, int kvh, int ntok, int warp,
+                                                 int lane)
+{
+    const int npp = kTile >> a.lp;
+    const int npg = (ntok + (1 << a.lp) - 1) >> a.lp;
+    const int mine = npg > warp ? (npg - warp + 3) >> 2 : 0;      // pages of this warp
+    if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(2 * mine * a.block_bytes));
+    __syncwarp();
+    if (lane < mine) {
+        const int j = warp + 4 * lane;
+        int pid = pids[j];
+        if (pid < 0 || pid >= a.num_pages) {
+            report_error(a.err, TQ_ERR_DEVICE_CHECK, kErrPageRange);
+            pid = 0;
+        }
+        const int64_t off = ((int64_t)pid * a.num_kv_heads + kvh) * a.block_bytes;
+        bulk_g2s(stage + j * a.block_bytes, a.kp + off, (uint32_t)a.block_bytes, bar);
+        bulk_g2s(stage + (npp + j) * a.block_bytes, a.vp + off, (uint32_t)a.block_bytes, bar);
+    }
+}
+
 // The split's page ids -> shared memory (at most 128: 2048 tokens of 16).
 __device__ __forceinline__ void load_split_pids(int* s_pid, const TcArgs& a, int b, int tok_begin,
                                                 int tok_end, int tid)
@@ -721,22 +746,35 @@ k_decode_tc(const TcArgs a)
 // ===================================================================
 // Integer tensor-core variant (kind::i8) for 2-, 4- and 8-bit codes.
 //
-//   S = K q''  A: K codes as unsigned bytes u (tensor memory, 32 columns);
-//              B: the scaled query q'' = rint(q' 2^s) as three balanced
-//              signed byte digits per row (column 4r + d); the accumulator
-//              starts at -L * sum(digits) so it holds sum (u - L) q'' exactly.
-//   O^T += V^T P''  A: V codes as signed bytes u - L (dim-major rows);
-//              B: P'' = rint(p s_v / L 2^(127 - ev) 2^22) as four unsigned
-//              byte digits per row.  O stays an exact int32 sum in tensor
-//              memory until the softmax rescales (rare) or the split ends,
-//              then it is folded into fp32 registers.
+//   S = K q''   A: K codes in tensor memory as unsigned bytes f_k u: a code
+//               keeps its bit position inside its byte (f_k = 1 or 16 for the
+//               low / high nibble of 4-bit codes; 1, 4, 16 or 64 for the
+//               four 2-bit fields), so unpacking costs one AND per word.
+//               B: (F / f_k) q'' with q'' = rint(q' 2^s) the fixed-point
+//               rotated query, as four balanced signed byte digits per row
+//               (column 4 r + d).  The accumulator starts at
+//               -L sum_k f_k B[k], so digit column d ends as the exact
+//               integer F sum_k (u_k - L) digit_d(q''_k) (|.| < 2^22).
+//   O^T += V^T P''  A: V codes as unsigned bytes u (dim-major rows).
+//               B: P'' = rint(p s_v / L 2^(127 - ev) 2^22) as four unsigned
+//               byte digits per row.  O holds sum_t u_t P''_t exactly in
+//               int32; the offset L sum_t P''_t is tracked exactly per row
+//               (64-bit) and taken off in 64-bit integers when O is folded
+//               into fp32 registers (on a rescale and at the end of the
+//               split), so the fold rounds once.
 // ===================================================================
 template <int BITS>
 struct I8Fmt {
     static constexpr int CB = 16 * BITS;
     static constexpr int L = (1 << (BITS - 1)) - 1;
+    static constexpr int F = BITS == 4 ? 16 : (BITS == 2 ? 64 : 1);
     static constexpr int kStage = 2 * kTile * (CB + 4);
 };
+
+// Shared-memory header of the integer kernel (bytes from the start).
+constexpr int kI8Pid = 1024;        // [128] split page ids
+constexpr int kI8Ps = 1536;         // [4][16] per-warp sums of P'' (u64)
+constexpr int kI8Hdr = 2048;        // operands and the ring follow
 
 // K position k of the byte operands -> dimension (K) or token (V)
 template <int BITS>
@@ -753,10 +791,32 @@ __device__ __forceinline__ int perm_i8_inv(int i)
     if constexpr (BITS == 2) return 16 * (i >> 4) + 4 * (i & 3) + ((i & 15) >> 2);
     return i;
 }
-
-// one word of codes -> unsigned bytes (u) in K-position order
+// in-place factor f_k of K position k
 template <int BITS>
-__device__ __forceinline__ void u8_of(uint32_t w, uint32_t* o)
+__device__ __forceinline__ int kfac_i8(int k)
+{
+    if constexpr (BITS == 4) return ((k >> 2) & 1) ? 16 : 1;
+    if constexpr (BITS == 2) return 1 << (2 * ((k >> 2) & 3));
+    return 1;
+}
+
+// K: one word of codes -> bytes f_k u (codes left in place)
+template <int BITS>
+__device__ __forceinline__ void k_bytes(uint32_t w, uint32_t* o)
+{
+    if constexpr (BITS == 4) {
+        o[0] = w & 0x0F0F0F0Fu;
+        o[1] = w & 0xF0F0F0F0u;
+    } else if constexpr (BITS == 2) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) o[j] = w & (0x03030303u << (2 * j));
+    } else {
+        o[0] = w;
+    }
+}
+// V: one word of codes -> bytes u
+template <int BITS>
+__device__ __forceinline__ void v_bytes(uint32_t w, uint32_t* o)
 {
     if constexpr (BITS == 4) {
         o[0] = w & 0x0F0F0F0Fu;
@@ -769,22 +829,6 @@ __device__ __forceinline__ void u8_of(uint32_t w, uint32_t* o)
     }
 }
 
-// bytes u -> signed bytes u - L, byte-wise without carries
-template <int BITS>
-__device__ __forceinline__ uint32_t s8_of(uint32_t u)
-{
-    if constexpr (BITS == 8) {
-        // (u + 129) mod 256 per byte
-        const uint32_t t = (u & 0x7F7F7F7Fu) + 0x01010101u;
-        uint32_t r;
-        asm("lop3.b32 %0, %1, %2, %3, 0xD2;" : "=r"(r) : "r"(t), "r"(u), "r"(0x80808080u));
-        return r;   // t ^ (~u & 0x80..): adds 128 + (u & 128) without a carry out
-    } else {
-        constexpr uint32_t Lb = (uint32_t)I8Fmt<BITS>::L * 0x01010101u;
-        return ((u | 0x80808080u) - Lb) ^ 0x80808080u;
-    }
-}
-
 template <int BITS>
 __device__ __forceinline__ void k_row_to_tmem_u8(const uint8_t* row, uint32_t taddr)
 {
@@ -794,15 +838,15 @@ __device__ __forceinline__ void k_row_to_tmem_u8(const uint8_t* row, uint32_t ta
         for (int h = 0; h < 2; ++h) {
             const uint4 a = *reinterpret_cast<const uint4*>(row + 32 * h);
             const uint4 b = *reinterpret_cast<const uint4*>(row + 32 * h + 16);
-            u8_of<4>(a.x, o); u8_of<4>(a.y, o + 2); u8_of<4>(a.z, o + 4); u8_of<4>(a.w, o + 6);
-            u8_of<4>(b.x, o + 8); u8_of<4>(b.y, o + 10); u8_of<4>(b.z, o + 12); u8_of<4>(b.w, o + 14);
+            k_bytes<4>(a.x, o); k_bytes<4>(a.y, o + 2); k_bytes<4>(a.z, o + 4); k_bytes<4>(a.w, o + 6);
+            k_bytes<4>(b.x, o + 8); k_bytes<4>(b.y, o + 10); k_bytes<4>(b.z, o + 12); k_bytes<4>(b.w, o + 14);
             tmem_st16(taddr + 16 * h, o);
         }
     } else if constexpr (BITS == 2) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const uint4 a = *reinterpret_cast<const uint4*>(row + 16 * h);
-            u8_of<2>(a.x, o); u8_of<2>(a.y, o + 4); u8_of<2>(a.z, o + 8); u8_of<2>(a.w, o + 12);
+            k_bytes<2>(a.x, o); k_bytes<2>(a.y, o + 4); k_bytes<2>(a.z, o + 8); k_bytes<2>(a.w, o + 12);
             tmem_st16(taddr + 16 * h, o);
         }
     } else {
@@ -819,10 +863,10 @@ __device__ __forceinline__ void k_row_to_tmem_u8(const uint8_t* row, uint32_t ta
 }
 
 // V codes of dimension `dim` for the tile's 128 tokens -> 32 words of
-// signed bytes in K-position order (registers; stored once the previous
+// unsigned bytes in K-position order (registers; stored once the previous
 // PV product has drained).
 template <int BITS>
-__device__ __forceinline__ void v_col_s8(const uint8_t* vblk0, int64_t bb, int lp, int dim,
+__device__ __forceinline__ void v_col_u8(const uint8_t* vblk0, int64_t bb, int lp, int dim,
                                          uint32_t* o)
 {
     const int P = 1 << lp;
@@ -833,8 +877,8 @@ __device__ __forceinline__ void v_col_s8(const uint8_t* vblk0, int64_t bb, int l
         const int t0 = 32 * q;
         const int pg = t0 >> lp, in = t0 & (P - 1);
         const uint8_t* row = vblk0 + pg * bb + (int64_t)dim * row_bytes;
-        uint32_t w[8];
         if constexpr (BITS == 4) {
+            uint32_t w[4];
             if (P >= 32) {
                 const uint4 x = *reinterpret_cast<const uint4*>(row + in / 2);
                 w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
@@ -844,13 +888,9 @@ __device__ __forceinline__ void v_col_s8(const uint8_t* vblk0, int64_t bb, int l
                 w[0] = x.x; w[1] = x.y; w[2] = y.x; w[3] = y.y;
             }
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                uint32_t u[2];
-                u8_of<4>(w[i], u);
-                o[8 * q + 2 * i] = s8_of<4>(u[0]);
-                o[8 * q + 2 * i + 1] = s8_of<4>(u[1]);
-            }
+            for (int i = 0; i < 4; ++i) v_bytes<4>(w[i], o + 8 * q + 2 * i);
         } else if constexpr (BITS == 2) {
+            uint32_t w[2];
             if (P >= 32) {
                 const uint2 x = *reinterpret_cast<const uint2*>(row + in / 4);
                 w[0] = x.x; w[1] = x.y;
@@ -858,13 +898,8 @@ __device__ __forceinline__ void v_col_s8(const uint8_t* vblk0, int64_t bb, int l
                 w[0] = *reinterpret_cast<const uint32_t*>(row);
                 w[1] = *reinterpret_cast<const uint32_t*>(row + bb);
             }
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                uint32_t u[4];
-                u8_of<2>(w[i], u);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) o[8 * q + 4 * i + j] = s8_of<2>(u[j]);
-            }
+            v_bytes<2>(w[0], o + 8 * q);
+            v_bytes<2>(w[1], o + 8 * q + 4);
         } else {
             uint4 x, y;
             if (P >= 32) {
@@ -874,10 +909,8 @@ __device__ __forceinline__ void v_col_s8(const uint8_t* vblk0, int64_t bb, int l
                 x = *reinterpret_cast<const uint4*>(row);
                 y = *reinterpret_cast<const uint4*>(row + bb);
             }
-            o[8 * q + 0] = s8_of<8>(x.x); o[8 * q + 1] = s8_of<8>(x.y);
-            o[8 * q + 2] = s8_of<8>(x.z); o[8 * q + 3] = s8_of<8>(x.w);
-            o[8 * q + 4] = s8_of<8>(y.x); o[8 * q + 5] = s8_of<8>(y.y);
-            o[8 * q + 6] = s8_of<8>(y.z); o[8 * q + 7] = s8_of<8>(y.w);
+            o[8 * q + 0] = x.x; o[8 * q + 1] = x.y; o[8 * q + 2] = x.z; o[8 * q + 3] = x.w;
+            o[8 * q + 4] = y.x; o[8 * q + 5] = y.y; o[8 * q + 6] = y.z; o[8 * q + 7] = y.w;
         }
     }
 }
@@ -892,13 +925,21 @@ __device__ __forceinline__ void umma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uin
                  : "memory");
 }
 
-// balanced signed byte digits of x (|x| < 2^22): x = d0 + 256 d1 + 65536 d2
-__device__ __forceinline__ void digits3(int x, int& d0, int& d1, int& d2)
+// balanced signed byte digits of x (|x| < 2^30): x = sum_d 256^d dd[d]
+__device__ __forceinline__ void digits4(int x, int* dd)
 {
-    d0 = (int)(int8_t)(x & 0xFF);
-    const int r1 = (x - d0) >> 8;
-    d1 = (int)(int8_t)(r1 & 0xFF);
-    d2 = (r1 - d1) >> 8;
+#pragma unroll
+    for (int d = 0; d < 3; ++d) {
+        dd[d] = (int)(int8_t)(x & 0xFF);
+        x = (x - dd[d]) >> 8;
+    }
+    dd[3] = x;
+}
+
+// exact int32 -> fp32 for |v| < 2^22 on the FP32/integer pipes
+__device__ __forceinline__ float small_int_to_float(uint32_t v)
+{
+    return __int_as_float((int)v + 0x4B400000) - 12582912.f;
 }
 
 template <int BITS, int RG>
@@ -909,10 +950,10 @@ k_decode_i8(const TcArgs a)
     constexpr int NS = 4 * RG;                       // S / O columns: 4r + digit
     constexpr uint32_t kColAK = 0, kColAV = 32, kColS = 64, kColO = 64 + NS;
     // kind::i8, s32 accumulate, M = 128, N = NS.  S: A u8, B s8 K-major.
-    // O: A s8, B u8 MN-major.
+    // O: A u8, B u8 MN-major.
     constexpr uint32_t kIdescS = (2u << 4) | (0u << 7) | (1u << 10) |
                                  ((uint32_t)(NS >> 3) << 17) | (8u << 24);
-    constexpr uint32_t kIdescO = (2u << 4) | (1u << 7) | (0u << 10) | (1u << 16) |
+    constexpr uint32_t kIdescO = (2u << 4) | (0u << 7) | (0u << 10) | (1u << 16) |
                                  ((uint32_t)(NS >> 3) << 17) | (8u << 24);
     constexpr uint32_t kQRow = (NS / 8) * 128;      // bytes per 16-deep K chunk of q''
     constexpr uint32_t kPRow = (NS / 16) * 128;     // bytes per 8-deep K group of P''
@@ -928,8 +969,9 @@ k_decode_i8(const TcArgs a)
     float* s_rowfac = reinterpret_cast<float*>(smem + 400);          // [16]
     float* s_l = reinterpret_cast<float*>(smem + 464);               // [4][16]
     int* s_init = reinterpret_cast<int*>(smem + 768);                // [NS] accumulator start
-    int* s_pid = reinterpret_cast<int*>(smem + 1024);                // [128] split page ids
-    uint8_t* s_qb = smem + 1536;                                     // q'' digits: 128 x NS bytes
+    int* s_pid = reinterpret_cast<int*>(smem + kI8Pid);
+    unsigned long long* s_ps = reinterpret_cast<unsigned long long*>(smem + kI8Ps);
+    uint8_t* s_qb = smem + kI8Hdr;                                   // q'' digits: 128 x NS bytes
     uint8_t* s_pb = s_qb + 128 * NS;                                 // P'' digits: 128 x NS bytes
     float* s_qf = reinterpret_cast<float*>(s_pb + 128 * NS);         // [RG][128] staging
     uint8_t* ring = reinterpret_cast<uint8_t*>(s_qf) + RG * 512;
@@ -955,7 +997,7 @@ k_decode_i8(const TcArgs a)
     const int npp = kTile >> a.lp;
 
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < kStages; ++s) mbar_init(&full[s], kTcThreads / 32);
         mbar_init(bar_s, 1);
         mbar_init(bar_o, 1);
         s_flag[0] = 0;
@@ -971,13 +1013,14 @@ k_decode_i8(const TcArgs a)
     const uint32_t tmem = *s_tmem;
     const uint32_t t_lane = tmem + ((uint32_t)(32 * warp) << 16);
 
-    if (warp == 0) {
-        for (int s = 0; s < kStages && s < ntiles; ++s) {
-            const int t0 = tok_begin + s * kTile;
-            issue_tile_tc(ring + s * F::kStage, &full[s], a,
-                          a.page_table + (int64_t)b * a.max_pages + (t0 >> a.lp), kvh,
-                          min(kTile, tok_end - t0), lane);
-        }
+    // bulk copies of a tile, shared by the 4 warps
+    auto issue_tile = [&](uint8_t* stg, uint64_t* bar, const int* pids, int t0) {
+        issue_tile_warps(stg, bar, a, pids, kvh, min(kTile, tok_end - t0), warp, lane);
+    };
+    for (int s = 0; s < kStages && s < ntiles; ++s) {
+        const int t0 = tok_begin + s * kTile;
+        issue_tile(ring + s * F::kStage, &full[s],
+                   a.page_table + (int64_t)b * a.max_pages + (t0 >> a.lp), t0);
     }
 
     load_split_pids(s_pid, a, b, tok_begin, tok_end, tid);   // visible after the next barrier
@@ -1009,72 +1052,70 @@ k_decode_i8(const TcArgs a)
         const float pre = pow2i(21 - ex);           // largest |q''| in [2^21, 2^22)
 #pragma unroll
         for (int e = 0; e < 4; ++e) s_qf[rr * kHeadDim + 4 * lane + e] = rintf(x[e] * pre);
-        if (lane == 0) s_rowfac[rr] = pow2i(ex - 21);
+        if (lane == 0) s_rowfac[rr] = pow2i(ex - 21) * (1.f / (float)F::F);
     }
     __syncthreads();
     {
-        // K position k = tid holds dimension perm(k); column 4r + d holds
-        // digit d of row r (d = 3: zero)
+        // K position k = tid holds dimension perm(k) with in-place factor f_k;
+        // column 4 r + d holds digit d of (F / f_k) q''_r
         const int k = tid;
         const int dim = perm_i8<BITS>(k);
-        int dsum[3 * RG];
+        const int fk = kfac_i8<BITS>(k);
+        int dsum[NS];
 #pragma unroll
         for (int r = 0; r < RG; ++r) {
-            int d0, d1, d2;
-            digits3((int)s_qf[r * kHeadDim + dim], d0, d1, d2);
-            const int dd[4] = {d0, d1, d2, 0};
+            int dd[4];
+            digits4((int)s_qf[r * kHeadDim + dim] * (F::F / fk), dd);
 #pragma unroll
             for (int d = 0; d < 4; ++d) {
                 const int n = 4 * r + d;
                 const int cm = (k >> 4) * (NS / 8) + (n >> 3);
                 s_qb[cm * 128 + (n & 7) * 16 + (k & 15)] = (uint8_t)(int8_t)dd[d];
-                if (d < 3) dsum[3 * r + d] = dd[d];
+                dsum[n] = fk * dd[d];
             }
         }
-        // accumulator start: -L * (sum over dims of each digit column), summed
-        // per warp by shuffles, then over the 4 warps in the (idle) P'' buffer
+        // accumulator start: -L sum_k f_k B[k][n], summed per warp by
+        // shuffles, then over the 4 warps in the (idle) P'' buffer
 #pragma unroll
-        for (int i = 0; i < 3 * RG; ++i) {
+        for (int i = 0; i < NS; ++i) {
             int v = dsum[i];
 #pragma unroll
             for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
             dsum[i] = v;
         }
-        int* s_sum = reinterpret_cast<int*>(s_pb);                   // [4][3 RG]
+        int* s_sum = reinterpret_cast<int*>(s_pb);                   // [4][NS]
         if (lane == 0)
 #pragma unroll
-            for (int i = 0; i < 3 * RG; ++i) s_sum[warp * 3 * RG + i] = dsum[i];
+            for (int i = 0; i < NS; ++i) s_sum[warp * NS + i] = dsum[i];
         __syncthreads();
         if (tid < NS) {
-            const int r = tid >> 2, d = tid & 3;
             int v = 0;
-            if (d < 3)
-                for (int w = 0; w < 4; ++w) v += s_sum[w * 3 * RG + 3 * r + d];
+            for (int w = 0; w < 4; ++w) v += s_sum[w * NS + tid];
             s_init[tid] = -F::L * v;
         }
     }
     float rowfac[RG];
-    int lim[RG];
 #pragma unroll
-    for (int r = 0; r < RG; ++r) {
-        rowfac[r] = s_rowfac[r];
-        const int R = rg * RG + r;
-        lim[r] = R < a.G ? seq_len - a.q_len + R / a.group : -1;
-    }
+    for (int r = 0; r < RG; ++r) rowfac[r] = s_rowfac[r];
     fence_proxy_async_smem();
     __syncthreads();
-    uint32_t sinit[NS];
+    // accumulator start of S: registers for 4 rows, re-read from shared
+    // memory for 8 (register pressure)
+    constexpr int kInitRegs = RG <= 4 ? NS : 1;
+    uint32_t sinit[kInitRegs];
 #pragma unroll
-    for (int n = 0; n < NS; ++n) sinit[n] = (uint32_t)s_init[n];
+    for (int n = 0; n < kInitRegs; ++n) sinit[n] = (uint32_t)s_init[n];
     const uint64_t desc_q = smem_desc(s_qb, kQRow, 128);
     const uint64_t desc_p = smem_desc(s_pb, kPRow, 128);
 
     float m_run[RG], l_run[RG], o_reg[RG];
+    unsigned long long psum[RG];        // this thread's tokens: sum of P'' since the last fold
 #pragma unroll
     for (int r = 0; r < RG; ++r) {
         m_run[r] = -CUDART_INF_F;
         l_run[r] = 0.f;
         o_reg[r] = 0.f;
+        psum[r] = 0ull;
     }
     int ev = 0;
     float vn = 1.f;
@@ -1085,7 +1126,18 @@ k_decode_i8(const TcArgs a)
     bool aborted = false;
     bool o_acc = false;                 // O holds an int32 sum to extend
 
-    // fold O (int32 digit sums, scale 2^(ev - 127) 2^-22) into o_reg (dimension tid)
+    // per-warp sums of psum -> s_ps (the caller synchronises before folding)
+    auto stash_psum = [&]() {
+#pragma unroll
+        for (int r = 0; r < RG; ++r) {
+            unsigned long long v = psum[r];
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
+            if (lane == 0) s_ps[warp * 16 + r] = v;
+        }
+    };
+    // fold O (sum u P'', int32 digits) minus L sum P'' into o_reg (dimension
+    // tid); scale_now = 2^(ev - 127) 2^-22
     auto flush_o = [&](float scale_now) {
         uint32_t ov[NS];
 #pragma unroll
@@ -1093,64 +1145,85 @@ k_decode_i8(const TcArgs a)
         tmem_wait_ld();
 #pragma unroll
         for (int r = 0; r < RG; ++r) {
-            float v = (float)(int)ov[4 * r + 3];
-            v = fmaf(v, 256.f, (float)(int)ov[4 * r + 2]);
-            v = fmaf(v, 256.f, (float)(int)ov[4 * r + 1]);
-            v = fmaf(v, 256.f, (float)(int)ov[4 * r]);
-            o_reg[r] = fmaf(v, scale_now, o_reg[r]);
+            const unsigned long long ps = s_ps[r] + s_ps[16 + r] + s_ps[32 + r] + s_ps[48 + r];
+            // digit sums are non-negative and below 2^31
+            const long long sum = (long long)ov[4 * r] + ((long long)ov[4 * r + 1] << 8) +
+                                  ((long long)ov[4 * r + 2] << 16) + ((long long)ov[4 * r + 3] << 24);
+            const long long v = sum - (long long)F::L * (long long)ps;
+            o_reg[r] = fmaf((float)v, scale_now, o_reg[r]);
+            psum[r] = 0ull;
         }
     };
 
-    for (int tt = 0; tt < ntiles; ++tt) {
-        const int stage = tt % kStages;
-        uint8_t* st = ring + stage * F::kStage;
-        const int tok0 = tok_begin + tt * kTile;
-        bool ok = mbar_wait_sleep(&full[stage], (uint32_t)((tt / kStages) & 1), kPollsTc);
-        tc_fence_after();
-        if (!ok) atomicOr(&s_flag[0], 1);
-
-        // K row of token tid -> A (u8); accumulator start -> S
+    // Software pipeline: S = K q'' of tile t + 1 is issued as soon as its K
+    // codes are in tensor memory, so it runs while tile t's softmax, V
+    // staging and PV product proceed; PV(t) drains while tile t + 1's
+    // scores are read and tile t + 2's K codes are staged.
+    //
+    // K codes of a tile -> A_K, accumulator start -> S, scales -> registers.
+    auto stage_k = [&](int t, float& ks_out, float& vs_out) {
+        const uint8_t* st = ring + (t % kStages) * F::kStage;
         const int pg = tid >> a.lp, row = tid & (P - 1);
         const uint8_t* kblk = st + pg * a.block_bytes;
         const uint8_t* vblk = st + (npp + pg) * a.block_bytes;
         k_row_to_tmem_u8<BITS>(kblk + row * F::CB, t_lane + kColAK);
+        if constexpr (RG <= 4) {
+            tmem_st16(t_lane + kColS, sinit);
+        } else {
 #pragma unroll
-        for (int c = 0; c < NS; c += 16) tmem_st16(t_lane + kColS + c, sinit + c);
-        float ks = reinterpret_cast<const float*>(kblk + P * F::CB)[row] * kinv;
-        float vs = reinterpret_cast<const float*>(vblk + P * F::CB)[row] * kinv;
-        const int tok = tok0 + tid;
-        if (tok >= tok_end) { ks = 0.f; vs = 0.f; }
+            for (int c = 0; c < NS; c += 16) {
+                uint32_t iv[16];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const uint4 x = reinterpret_cast<const uint4*>(s_init + c)[q4];
+                    iv[4 * q4] = x.x; iv[4 * q4 + 1] = x.y; iv[4 * q4 + 2] = x.z; iv[4 * q4 + 3] = x.w;
+                }
+                tmem_st16(t_lane + kColS + c, iv);
+            }
+        }
+        ks_out = reinterpret_cast<const float*>(kblk + P * F::CB)[row] * kinv;
+        vs_out = reinterpret_cast<const float*>(vblk + P * F::CB)[row] * kinv;
+        if (tok_begin + t * kTile + tid >= tok_end) { ks_out = 0.f; vs_out = 0.f; }
+    };
+    auto issue_qk = [&]() {
+        tc_fence_after();
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            umma_i8_ts(tmem + kColS, tmem + kColAK + 8 * j, desc_q + ((2 * j * kQRow) >> 4), kIdescS,
+                       1u);
+        umma_commit(bar_s);
+    };
+
+    float ks, vs;                       // scales of the tile whose scores come next
+    {
+        bool ok = mbar_wait_sleep(&full[0], 0u, kPollsTc);
+        tc_fence_after();
+        if (!ok) atomicOr(&s_flag[0], 1);
+        stage_k(0, ks, vs);
         tmem_wait_st();
         tc_fence_before();
         __syncthreads();
-        if (s_flag[0]) { aborted = true; break; }
+        if (s_flag[0]) aborted = true;
+        else if (tid == 0) issue_qk();
+    }
 
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                umma_i8_ts(tmem + kColS, tmem + kColAK + 8 * j, desc_q + ((2 * j * kQRow) >> 4),
-                           kIdescS, 1u);
-            umma_commit(bar_s);
-        }
+    for (int tt = 0; tt < ntiles && !aborted; ++tt) {
+        const int stage = tt % kStages;
+        uint8_t* st = ring + stage * F::kStage;
+        const int tok0 = tok_begin + tt * kTile;
+        const int tok = tok0 + tid;
 
-        // V column of dimension tid (registers) while S is computed
-        uint32_t vw[32];
-        v_col_s8<BITS>(st + npp * a.block_bytes, a.block_bytes, a.lp, tid, vw);
-        if (tt > 0) {
-            ok = mbar_wait_sleep(bar_o, (uint32_t)((tt - 1) & 1), kPollsTc);
-            tc_fence_after();
-            if (!ok) atomicOr(&s_flag[0], 1);
-        }
-        tmem_st16(t_lane + kColAV, vw);
-        tmem_st16(t_lane + kColAV + 16, vw + 16);
-
-        ok = mbar_wait_sleep(bar_s, (uint32_t)(tt & 1), kPollsTc);
+        // a. scores of tile tt
+        bool ok = mbar_wait_sleep(bar_s, (uint32_t)(tt & 1), kPollsTc);
         tc_fence_after();
-        if (!ok) atomicOr(&s_flag[0], 1);
         uint32_t sraw[NS];
 #pragma unroll
         for (int c = 0; c < NS; c += 16) tmem_ld16(t_lane + kColS + c, sraw + c);
+
+        // b. V column of dimension tid (registers), overlapping the load of
+        // S for 4 rows; after the scores for 8 (register pressure)
+        uint32_t vw[32];
+        if constexpr (RG <= 4) v_col_u8<BITS>(st + npp * a.block_bytes, a.block_bytes, a.lp, tid, vw);
         tmem_wait_ld();
 
         const bool full_tile = tok0 + kTile - 1 <= lim_min;
@@ -1158,21 +1231,51 @@ k_decode_i8(const TcArgs a)
         bool need = false;
 #pragma unroll
         for (int r = 0; r < RG; ++r) {
-            float v = fmaf((float)(int)sraw[4 * r + 2], 65536.f, (float)(int)sraw[4 * r + 1] * 256.f);
-            v += (float)(int)sraw[4 * r];
+            float v = small_int_to_float(sraw[4 * r + 1]) * 256.f + small_int_to_float(sraw[4 * r]);
+            v = fmaf(small_int_to_float(sraw[4 * r + 2]), 65536.f, v);
+            if constexpr (BITS != 8) v = fmaf(small_int_to_float(sraw[4 * r + 3]), 16777216.f, v);
             float x = v * (ks * rowfac[r]);
-            if (!full_tile) x = tok <= lim[r] ? x : -CUDART_INF_F;
+            if (!full_tile) {
+                const int R = rg * RG + r;
+                const int lr = R < a.G ? seq_len - a.q_len + R / a.group : -1;
+                x = tok <= lr ? x : -CUDART_INF_F;
+            }
             sc[r] = x;
             need |= x > m_run[r] + kLazyTc;
         }
         need |= vs >= vlimit;
+        const float vs_t = vs;
+        if constexpr (RG > 4) v_col_u8<BITS>(st + npp * a.block_bytes, a.block_bytes, a.lp, tid, vw);
+
+        // c. K codes of tile tt + 1 (S of tile tt is in registers)
+        if (tt + 1 < ntiles) {
+            ok = ok && mbar_wait_sleep(&full[(tt + 1) % kStages], (uint32_t)(((tt + 1) / kStages) & 1),
+                                       kPollsTc);
+            tc_fence_after();
+            stage_k(tt + 1, ks, vs);
+        }
+
+        // d. PV(tt - 1) has drained: A_V, O and the P'' buffer are free
+        if (tt > 0) {
+            ok = ok && mbar_wait_sleep(bar_o, (uint32_t)((tt - 1) & 1), kPollsTc);
+            tc_fence_after();
+        }
+        if (!ok) atomicOr(&s_flag[0], 1);
+        tmem_st16(t_lane + kColAV, vw);
+        tmem_st16(t_lane + kColAV + 16, vw + 16);
+        tmem_wait_st();
+        tc_fence_before();
+
+        // e. one barrier: tile tt + 1's operands are staged, stage tt is consumed
         const int any = __syncthreads_or(need);
         if (s_flag[0]) { aborted = true; break; }
-        if (warp == 0 && tt + kStages < ntiles) {
+        if (tid == 0 && tt + 1 < ntiles) issue_qk();
+        if (tt + kStages < ntiles) {
             const int t0 = tok_begin + (tt + kStages) * kTile;
-            issue_tile_tc(st, &full[stage], a, s_pid + ((t0 - tok_begin) >> a.lp), kvh,
-                          min(kTile, tok_end - t0), lane);
+            issue_tile(st, &full[stage], s_pid + ((t0 - tok_begin) >> a.lp), t0);
         }
+
+        // f. rare: new row maxima or a larger V scale exponent
         if (any) {
 #pragma unroll
             for (int r = 0; r < RG; ++r) {
@@ -1181,10 +1284,10 @@ k_decode_i8(const TcArgs a)
                 for (int m = 16; m >= 1; m >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, m));
                 if (lane == 0) s_red[warp * 16 + r] = v;
             }
-            const unsigned vb = __reduce_max_sync(kFull, __float_as_uint(vs));
+            const unsigned vb = __reduce_max_sync(kFull, __float_as_uint(vs_t));
             if (lane == 0) s_redv[warp] = vb;
+            if (o_acc) stash_psum();
             __syncthreads();
-            // fold the running int32 O (old scale) into o_reg, then rescale
             if (o_acc) flush_o(pow2i(ev - 127 - 22));
             o_acc = false;
             const unsigned vmax = max(max(s_redv[0], s_redv[1]), max(s_redv[2], s_redv[3]));
@@ -1201,11 +1304,12 @@ k_decode_i8(const TcArgs a)
                 l_run[r] *= alpha;
                 o_reg[r] *= alpha;
             }
+            tc_fence_before();
             __syncthreads();
         }
 
-        // P'' row of token tid at K position kpos: 4 digit bytes per row
-        const float vn_t = vs * vn * 4194304.f;       // 2^22 fixed point
+        // g. P'' row of token tid at K position kpos: 4 digit bytes per row
+        const float vn_t = vs_t * vn * 4194304.f;       // 2^22 fixed point
         uint32_t pw[RG];
 #pragma unroll
         for (int r = 0; r < RG; ++r) {
@@ -1213,6 +1317,7 @@ k_decode_i8(const TcArgs a)
             if (!full_tile) pr = sc[r] == -CUDART_INF_F ? 0.f : pr;
             l_run[r] += pr;
             pw[r] = pr > 0.f ? __float2uint_rn(pr * vn_t) : 0u;
+            psum[r] += pw[r];
         }
         {
             uint8_t* rowp = s_pb + (kpos >> 3) * kPRow + (kpos & 7) * 16;
@@ -1221,10 +1326,10 @@ k_decode_i8(const TcArgs a)
                 *reinterpret_cast<uint4*>(rowp + ng * 128) =
                     make_uint4(pw[4 * ng], pw[4 * ng + 1], pw[4 * ng + 2], pw[4 * ng + 3]);
         }
-        tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
+        // h. O^T += V^T P''
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
@@ -1239,12 +1344,11 @@ k_decode_i8(const TcArgs a)
     // ---- epilogue
     bool ok = !aborted && mbar_wait_sleep(bar_o, (uint32_t)((ntiles - 1) & 1), kPollsTc);
     tc_fence_after();
+    ok = __syncthreads_and(ok);
     const int nrows = min(RG, a.G - rg * RG);
     float* sO = reinterpret_cast<float*>(ring);          // [RG][128]
     if (ok) {
-        if (o_acc) flush_o(pow2i(ev - 127 - 22));
-#pragma unroll
-        for (int r = 0; r < RG; ++r) sO[r * kHeadDim + tid] = o_reg[r];
+        stash_psum();
 #pragma unroll
         for (int r = 0; r < RG; ++r) {
             float l = l_run[r];
@@ -1252,6 +1356,10 @@ k_decode_i8(const TcArgs a)
             for (int m = 16; m >= 1; m >>= 1) l += __shfl_xor_sync(kFull, l, m);
             if (lane == 0) s_l[warp * 16 + r] = l;
         }
+        __syncthreads();
+        if (o_acc) flush_o(pow2i(ev - 127 - 22));
+#pragma unroll
+        for (int r = 0; r < RG; ++r) sO[r * kHeadDim + tid] = o_reg[r];
     } else if (tid == 0) {
         report_error(a.err, TQ_ERR_TIMEOUT, kErrWaitTile);
     }
@@ -1288,7 +1396,7 @@ template <int BITS, int RG>
 cudaError_t launch_i8(const TcArgs& a, dim3 grid, cudaStream_t stream)
 {
     constexpr int NS = 4 * RG;
-    const size_t smem = 1536 + 2 * 128 * NS + RG * 512 + (size_t)kStages * I8Fmt<BITS>::kStage;
+    const size_t smem = kI8Hdr + 2 * 128 * NS + RG * 512 + (size_t)kStages * I8Fmt<BITS>::kStage;
     static int configured = 0;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
