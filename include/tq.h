@@ -27,7 +27,11 @@
  * Cache layout in device memory (one pool for K, one for V, same shape):
  *   pool[num_pages][num_kv_heads][block], block = tq_page_block_bytes(...).
  *   turbo b-bit K block: page_size token rows of d*b/8 code bytes (row t =
- *   token t's packed vector), then page_size fp32 scales.
+ *   token t's packed vector), then page_size fp32 scales.  For b = 2, 4, 8
+ *   the 16-byte chunks of row t are permuted: logical chunk c is stored at
+ *   chunk c ^ w(t), with w(t) = (t >> 2) & 1, (t >> 1) & 3, t & 7 for
+ *   b = 2, 4, 8 (a bank-conflict-free read pattern); 3-bit rows are stored
+ *   in order.
  *   turbo b-bit V block: the same codes dim-major -- d rows of
  *   page_size*b/8 bytes, row i holding every token's code i (token t at bits
  *   [t*b, (t+1)*b) of the row, LSB-first) -- then page_size fp32 scales.

@@ -43,8 +43,9 @@ __device__ __forceinline__ void fwht128_lane(float x[4], int lane)
 }
 
 template <int BITS>
-__device__ __forceinline__ void store_codes(uint8_t* dst, const uint32_t u[4], int lane)
+__device__ __forceinline__ void store_codes(uint8_t* dst, const uint32_t u[4], int lane, int sw)
 {
+    // the lane holding chunk c stores it at chunk c ^ sw (sw = 0 for 3 bits)
     // piece = this lane's 4 codes, LSB-first: code e at bits [e*BITS, (e+1)*BITS)
     uint32_t piece = u[0] | (u[1] << BITS) | (u[2] << (2 * BITS)) | (u[3] << (3 * BITS));
     if constexpr (BITS == 8) {
@@ -53,7 +54,7 @@ __device__ __forceinline__ void store_codes(uint8_t* dst, const uint32_t u[4], i
 #pragma unroll
         for (int k = 0; k < 4; ++k) w[k] = __shfl_sync(kFull, piece, 4 * (lane & 7) + k);
         if (lane < 8)
-            *reinterpret_cast<uint4*>(dst + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(dst + 16 * (lane ^ sw)) = make_uint4(w[0], w[1], w[2], w[3]);
     } else if constexpr (BITS == 4) {
         uint32_t nb = __shfl_down_sync(kFull, piece, 1);
         uint32_t word = piece | (nb << 16);          // valid on even lanes: word lane/2
@@ -61,7 +62,7 @@ __device__ __forceinline__ void store_codes(uint8_t* dst, const uint32_t u[4], i
 #pragma unroll
         for (int k = 0; k < 4; ++k) w[k] = __shfl_sync(kFull, word, 8 * (lane & 3) + 2 * k);
         if (lane < 4)
-            *reinterpret_cast<uint4*>(dst + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(dst + 16 * (lane ^ sw)) = make_uint4(w[0], w[1], w[2], w[3]);
     } else if constexpr (BITS == 2) {
         uint32_t half = piece | (__shfl_down_sync(kFull, piece, 1) << 8);
         uint32_t word = half | (__shfl_down_sync(kFull, half, 2) << 16);  // lanes 4w
@@ -69,7 +70,7 @@ __device__ __forceinline__ void store_codes(uint8_t* dst, const uint32_t u[4], i
 #pragma unroll
         for (int k = 0; k < 4; ++k) w[k] = __shfl_sync(kFull, word, 16 * (lane & 1) + 4 * k);
         if (lane < 2)
-            *reinterpret_cast<uint4*>(dst + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(dst + 16 * (lane ^ sw)) = make_uint4(w[0], w[1], w[2], w[3]);
     } else {  // BITS == 3: 12-bit pieces, 48 bytes per vector
         // 24-bit groups (8 codes) on even lanes: group lane/2 at bit 24*(lane/2)
         uint32_t grp = piece | (__shfl_down_sync(kFull, piece, 1) << 12);
@@ -186,7 +187,7 @@ k_quantize_append(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v
     uint8_t* blk = (which ? vp : kp) + (page * num_kv_heads + head) * block_bytes;
     if (!which) {
         // K: the packed vector is token row `off`
-        store_codes<BITS>(blk + (int64_t)off * CB, u, lane);
+        store_codes<BITS>(blk + (int64_t)off * CB, u, lane, k_swizzle<BITS>(off));
     } else {
         // V: dim-major rows; code i is field `off` of row i
         store_dim_major<BITS>(blk, u, lane, off, page_size);

@@ -947,17 +947,7 @@ cudaError_t launch_decode(const void* q, const tq_cache& c, int64_t block_bytes,
     }
     const dim3 grid((unsigned)a.max_splits, (unsigned)(c.num_kv_heads * a.R), (unsigned)batch);
     const bool two = (a.G > 4);   // more than 4 rows in a row group
-#define TQ_DEC(B)                                                                      \
-    return two ? launch_one<B, 2>(a, grid, stream) : launch_one<B, 1>(a, grid, stream)
-    switch (c.format) {
-    case 2: TQ_DEC(2);
-    case 3: TQ_DEC(3);
-    case 4: TQ_DEC(4);
-    case 8: TQ_DEC(8);
-    case 16: TQ_DEC(16);
-    default: return cudaErrorInvalidValue;
-    }
-#undef TQ_DEC
+    return two ? launch_one<16, 2>(a, grid, stream) : launch_one<16, 1>(a, grid, stream);
 }
 
 }  // namespace tq

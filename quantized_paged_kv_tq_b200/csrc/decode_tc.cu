@@ -829,15 +829,18 @@ __device__ __forceinline__ void v_bytes(uint32_t w, uint32_t* o)
     }
 }
 
+// K row of one token (its chunks permuted by `sw`, see k_swizzle) -> bytes
+// f_k u in tensor memory columns [0, 32) of this thread's lane.
 template <int BITS>
-__device__ __forceinline__ void k_row_to_tmem_u8(const uint8_t* row, uint32_t taddr)
+__device__ __forceinline__ void k_row_to_tmem_u8(const uint8_t* row, uint32_t taddr, int sw)
 {
     uint32_t o[16];
+    auto chunk = [&](int c) { return *reinterpret_cast<const uint4*>(row + 16 * (c ^ sw)); };
     if constexpr (BITS == 4) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            const uint4 a = *reinterpret_cast<const uint4*>(row + 32 * h);
-            const uint4 b = *reinterpret_cast<const uint4*>(row + 32 * h + 16);
+            const uint4 a = chunk(2 * h);
+            const uint4 b = chunk(2 * h + 1);
             k_bytes<4>(a.x, o); k_bytes<4>(a.y, o + 2); k_bytes<4>(a.z, o + 4); k_bytes<4>(a.w, o + 6);
             k_bytes<4>(b.x, o + 8); k_bytes<4>(b.y, o + 10); k_bytes<4>(b.z, o + 12); k_bytes<4>(b.w, o + 14);
             tmem_st16(taddr + 16 * h, o);
@@ -845,7 +848,7 @@ __device__ __forceinline__ void k_row_to_tmem_u8(const uint8_t* row, uint32_t ta
     } else if constexpr (BITS == 2) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            const uint4 a = *reinterpret_cast<const uint4*>(row + 16 * h);
+            const uint4 a = chunk(h);
             k_bytes<2>(a.x, o); k_bytes<2>(a.y, o + 4); k_bytes<2>(a.z, o + 8); k_bytes<2>(a.w, o + 12);
             tmem_st16(taddr + 16 * h, o);
         }
@@ -854,7 +857,7 @@ __device__ __forceinline__ void k_row_to_tmem_u8(const uint8_t* row, uint32_t ta
         for (int h = 0; h < 2; ++h) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const uint4 a = *reinterpret_cast<const uint4*>(row + 64 * h + 16 * q);
+                const uint4 a = chunk(4 * h + q);
                 o[4 * q] = a.x; o[4 * q + 1] = a.y; o[4 * q + 2] = a.z; o[4 * q + 3] = a.w;
             }
             tmem_st16(taddr + 16 * h, o);
@@ -1166,7 +1169,7 @@ k_decode_i8(const TcArgs a)
         const int pg = tid >> a.lp, row = tid & (P - 1);
         const uint8_t* kblk = st + pg * a.block_bytes;
         const uint8_t* vblk = st + (npp + pg) * a.block_bytes;
-        k_row_to_tmem_u8<BITS>(kblk + row * F::CB, t_lane + kColAK);
+        k_row_to_tmem_u8<BITS>(kblk + row * F::CB, t_lane + kColAK, k_swizzle<BITS>(row));
         if constexpr (RG <= 4) {
             tmem_st16(t_lane + kColS, sinit);
         } else {
@@ -1185,6 +1188,9 @@ k_decode_i8(const TcArgs a)
         vs_out = reinterpret_cast<const float*>(vblk + P * F::CB)[row] * kinv;
         if (tok_begin + t * kTile + tid >= tok_end) { ks_out = 0.f; vs_out = 0.f; }
     };
+    // One thread issues the 4 K-steps of a product and commits them: MMAs
+    // accumulating into one tensor-memory accumulator stay in one thread's
+    // issue order.
     auto issue_qk = [&]() {
         tc_fence_after();
 #pragma unroll
@@ -1193,6 +1199,22 @@ k_decode_i8(const TcArgs a)
                        1u);
         umma_commit(bar_s);
     };
+    auto issue_pv = [&]() {
+        tc_fence_after();
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            umma_i8_ts(tmem + kColO, tmem + kColAV + 8 * j, desc_p + ((4 * j * kPRow) >> 4),
+                       kIdescO, 1u);
+        umma_commit(bar_o);
+    };
+    // O starts (and restarts after each fold) at zero: every PV step accumulates
+    auto zero_o = [&]() {
+        uint32_t z[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) z[i] = 0u;
+#pragma unroll
+        for (int c = 0; c < NS; c += 16) tmem_st16(t_lane + kColO + c, z);
+    };
 
     float ks, vs;                       // scales of the tile whose scores come next
     {
@@ -1200,6 +1222,7 @@ k_decode_i8(const TcArgs a)
         tc_fence_after();
         if (!ok) atomicOr(&s_flag[0], 1);
         stage_k(0, ks, vs);
+        zero_o();
         tmem_wait_st();
         tc_fence_before();
         __syncthreads();
@@ -1288,7 +1311,11 @@ k_decode_i8(const TcArgs a)
             if (lane == 0) s_redv[warp] = vb;
             if (o_acc) stash_psum();
             __syncthreads();
-            if (o_acc) flush_o(pow2i(ev - 127 - 22));
+            if (o_acc) {
+                flush_o(pow2i(ev - 127 - 22));
+                zero_o();
+                tmem_wait_st();
+            }
             o_acc = false;
             const unsigned vmax = max(max(s_redv[0], s_redv[1]), max(s_redv[2], s_redv[3]));
             ev = max(ev, (int)(vmax >> 23));
@@ -1330,14 +1357,7 @@ k_decode_i8(const TcArgs a)
         tc_fence_before();
         __syncthreads();
         // h. O^T += V^T P''
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                umma_i8_ts(tmem + kColO, tmem + kColAV + 8 * j, desc_p + ((4 * j * kPRow) >> 4),
-                           kIdescO, (o_acc || j > 0) ? 1u : 0u);
-            umma_commit(bar_o);
-        }
+        if (tid == 0) issue_pv();
         o_acc = true;
     }
 

@@ -77,6 +77,17 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
     return ok != 0;
 }
 
+// K token rows are stored with their 16-byte chunks permuted: chunk c of the
+// row at offset r in its page sits at chunk c ^ k_swizzle<BITS>(r).  Eight
+// consecutive rows then hold a given chunk in eight different 16-byte bank
+// groups, so a thread per token reads its row without bank conflicts.
+// 3-bit rows (48 bytes) are stored as they are.
+template <int BITS>
+__host__ __device__ constexpr int k_swizzle(int r)
+{
+    return BITS == 4 ? (r >> 1) & 3 : (BITS == 2 ? (r >> 2) & 1 : (BITS == 8 ? r & 7 : 0));
+}
+
 // Non-blocking test of a phase.
 __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity)
 {

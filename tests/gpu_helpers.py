@@ -109,6 +109,29 @@ def check_close(got: np.ndarray, ref: np.ndarray, what: str = "") -> dict:
     return {"max_abs": max_abs, "rel_l2": rel_l2}
 
 
+def k_unswizzle(rows: np.ndarray, off: int, fmt: int) -> np.ndarray:
+    """Undo the documented 16-byte chunk permutation of a K token row at
+    offset `off` in its page (include/tq.h: logical chunk c is stored at
+    chunk c ^ w(off))."""
+    w = {2: (off >> 2) & 1, 4: (off >> 1) & 3, 8: off & 7}.get(fmt, 0)
+    if w == 0:
+        return rows
+    n = rows.shape[-1] // 16
+    chunks = rows.reshape(rows.shape[:-1] + (n, 16))
+    return chunks[..., [c ^ w for c in range(n)], :].reshape(rows.shape)
+
+
+def k_pool_logical(kp: np.ndarray, fmt: int, P: int) -> np.ndarray:
+    """A K pool [pages][heads][block] with every token row's chunk
+    permutation undone (token rows in plain packed order, scales as they
+    are)."""
+    out = kp.copy()
+    cb = 128 * fmt // 8
+    for r in range(P):
+        out[..., r * cb:(r + 1) * cb] = k_unswizzle(kp[..., r * cb:(r + 1) * cb], r, fmt)
+    return out
+
+
 def gpu_rows(cache: tq.Cache, slots: np.ndarray, P: int, fmt: int):
     """K packed rows, V offset-binary values (read from the dim-major V
     block) and the fp32 scales of K and V at `slots` (host copy)."""
@@ -118,7 +141,8 @@ def gpu_rows(cache: tq.Cache, slots: np.ndarray, P: int, fmt: int):
     vb = cache.v_pages[pages].cpu().numpy()
     cb = 128 * fmt // 8
     idx = np.arange(len(slots))
-    kc = np.stack([kb[i, :, offs[i] * cb:(offs[i] + 1) * cb] for i in idx])
+    kc = np.stack([k_unswizzle(kb[i, :, offs[i] * cb:(offs[i] + 1) * cb], int(offs[i]), fmt)
+                   for i in idx])
     vbits = np.unpackbits(vb[:, :, :P * cb], axis=-1, bitorder="little")
     vbits = vbits.reshape(len(slots), vb.shape[1], 128, P, fmt)[idx, :, :, offs]
     vu = (vbits * (1 << np.arange(fmt))).sum(-1)

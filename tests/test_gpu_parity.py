@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import oracle
-from gpu_helpers import (check_close, dev, dev_bf16, gpu_decode, gpu_fill, gpu_rows,
+from gpu_helpers import (check_close, dev, dev_bf16, gpu_decode, gpu_fill, gpu_rows, k_pool_logical,
                          oracle_decode, oracle_pools, oracle_rows)
 from quantized_paged_kv_tq_b200 import workloads as W
 
@@ -42,7 +42,7 @@ def test_quantize_append_bit_exact_small(fmt, P):
     kp, vp = oracle_pools(fmt, w.num_pages, w)
     for slots, k, v in w.iter_fill():
         oracle.quantize_append(k, v, slots, fmt, P, kp, vp)
-    assert np.array_equal(cache.k_pages.cpu().numpy(), kp)
+    assert np.array_equal(k_pool_logical(cache.k_pages.cpu().numpy(), fmt, P), kp)
     assert np.array_equal(cache.v_pages.cpu().numpy(), vp)
     assert cache.read_error() == 0
 
@@ -68,7 +68,7 @@ def test_quantize_special_vectors(fmt):
     torch.cuda.synchronize()
     kp, vp = oracle_pools(fmt, 2, W.custom(num_kv_heads=2, page_size=16))
     oracle.quantize_append(k, v, slots, fmt, 16, kp, vp)
-    assert np.array_equal(cache.k_pages.cpu().numpy(), kp)
+    assert np.array_equal(k_pool_logical(cache.k_pages.cpu().numpy(), fmt, 16), kp)
     assert np.array_equal(cache.v_pages.cpu().numpy(), vp)
 
 
