@@ -45,6 +45,24 @@ DEFAULT_WORKLOAD = "target64x8k"
 FALLBACK_HBM_GBS = 6650.0
 
 
+def max_over_ranks(times, world: int, device=None):
+    """Element-wise maximum of per-rank times (all ranks call it in the same
+    order; a no-op for one rank)."""
+    if world <= 1:
+        return list(times)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(times), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(bytes_per_rank_step: int, world: int, ms_step: float) -> float:
+    """Whole-job GB/s: every rank's bytes over the slowest rank's step time
+    (replicas with the same per-rank workload: weak scaling)."""
+    return world * bytes_per_rank_step / (ms_step * 1e-3) / 1e9
+
+
 def describe(w: W.Workload, fmt: int) -> str:
     names = {2: "turbo2", 3: "turbo3", 4: "turbo4", 8: "turbo8", 16: "bf16"}
     lens = (f"{int(w.seq_lens[0])} tokens" if np.all(w.seq_lens == w.seq_lens[0])
@@ -402,18 +420,13 @@ def run_ours(args):
         raise SystemExit(f"device error word set: 0x{err:x}")
 
     # ---- reduce over ranks: max of each time
-    ms_step = total_ms / K
-    dec_avg = sum(decode_ms) / K
-    app_avg = sum(append_ms) / K
-    if world > 1:
-        t = torch.tensor([ms_step, dec_avg, app_avg, e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, dec_avg, app_avg, e2e_ms = t.tolist()
+    ms_step, dec_avg, app_avg, e2e_ms = max_over_ranks(
+        [total_ms / K, sum(decode_ms) / K, sum(append_ms) / K, e2e_ms], world, dev)
 
     kv_bytes, app_bytes = step_bytes(w, fmt)
     peaks, peak_kind = measured_peaks()
     peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
-    value = world * kv_bytes / (ms_step * 1e-3) / 1e9
+    value = job_throughput(kv_bytes, world, ms_step)
     achieved = kv_bytes / (dec_avg * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
