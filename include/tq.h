@@ -24,8 +24,10 @@
  *             Query position t of q_len sees keys j <= seq_len - q_len + t.
  *             Query head h reads kv head h / (num_q_heads / num_kv_heads).
  *
- * Cache layout in device memory (one pool for K, one for V, same shape):
- *   pool[num_pages][num_kv_heads][block], block = tq_page_block_bytes(...).
+ * Cache layout in device memory (one pool per layer):
+ *   pool[num_pages][num_kv_heads][2][block], block = tq_page_block_bytes(...):
+ *   the K block, then the V block, of each (page, kv head).  K and V of a
+ *   page are adjacent so that decode fetches both with one bulk copy.
  *   turbo b-bit K block: page_size token rows of d*b/8 code bytes (row t =
  *   token t's packed vector), then page_size fp32 scales.  For b = 2, 4, 8
  *   the 16-byte chunks of row t are permuted: logical chunk c is stored at
@@ -68,7 +70,7 @@
 extern "C" {
 #endif
 
-#define TQ_ABI_VERSION 1
+#define TQ_ABI_VERSION 2
 
 typedef enum {
     TQ_OK = 0,
@@ -90,16 +92,16 @@ typedef enum {
     TQ_BF16 = 16
 } tq_format;
 
-/* Descriptor of one layer's paged K/V pools.  Plain data; the pointed-to
+/* Descriptor of one layer's paged K/V pool.  Plain data; the pointed-to
  * device memory is owned by the caller. */
 typedef struct {
     int32_t format;        /* tq_format */
     int32_t head_dim;      /* d; must be 128 */
     int32_t num_kv_heads;  /* >= 1 */
     int32_t page_size;     /* tokens per page: 16, 32 or 64 */
-    int32_t num_pages;     /* pages in each pool, >= 1 */
-    void* k_pages;         /* device, 16-byte aligned, num_pages*num_kv_heads*block bytes */
-    void* v_pages;         /* device, same size and alignment */
+    int32_t num_pages;     /* pages in the pool, >= 1 */
+    void* pages;           /* device, 16-byte aligned, num_pages*num_kv_heads*2*block bytes:
+                              [page][kv head][K block, V block] */
     uint32_t* dev_error;   /* device word, optional (NULL: device findings dropped).
                               0 = no error; else (tq_status) | (detail << 8). */
 } tq_cache;
@@ -110,8 +112,9 @@ int32_t tq_abi_version(void);
 /* Readable name of a status.  Never NULL; the string is static. */
 const char* tq_status_string(tq_status status);
 
-/* Bytes of one (page, kv head) block of a pool, per the layout above; 0 when
- * the arguments are not a supported combination. */
+/* Bytes of one K (or V) block of one (page, kv head), per the layout above
+ * (the pool holds num_pages * num_kv_heads * 2 of them); 0 when the arguments
+ * are not a supported combination. */
 size_t tq_page_block_bytes(int32_t format, int32_t head_dim, int32_t page_size);
 
 /*
@@ -126,7 +129,7 @@ size_t tq_page_block_bytes(int32_t format, int32_t head_dim, int32_t page_size);
  *   num_tokens    >= 0 (0 is a no-op).
  *   bits          2, 3, 4 or 8; must equal cache->format.
  * Result: codes and the fp32 scale of every (token, head) of K and of V are
- * written at their slot; nothing else in the pools changes.  Bit-exact with
+ * written at their slot; nothing else in the pool changes.  Bit-exact with
  * the definition above for every finite input.
  */
 tq_status tq_quantize_append(const void* k, const void* v,

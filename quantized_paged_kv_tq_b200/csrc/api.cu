@@ -66,8 +66,7 @@ tq_status check_cache(const tq_cache* c, bool want_turbo)
         return TQ_ERR_INVALID_ARG;
     if (c->head_dim != 128) return TQ_ERR_UNSUPPORTED;
     if (c->page_size != 16 && c->page_size != 32 && c->page_size != 64) return TQ_ERR_UNSUPPORTED;
-    if (!c->k_pages || !c->v_pages) return TQ_ERR_INVALID_ARG;
-    if (!aligned16(c->k_pages) || !aligned16(c->v_pages)) return TQ_ERR_INVALID_ARG;
+    if (!c->pages || !aligned16(c->pages)) return TQ_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(c->dev_error) & 3u) != 0) return TQ_ERR_INVALID_ARG;
     return TQ_OK;
 }

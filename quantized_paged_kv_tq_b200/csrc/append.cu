@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(32 * kAppendWarps)
 k_quantize_append(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
                   const int64_t* __restrict__ slots, int num_tokens, int num_kv_heads,
                   int page_size, int num_pages, int64_t block_bytes,
-                  uint8_t* __restrict__ kp, uint8_t* __restrict__ vp, uint32_t* err)
+                  uint8_t* __restrict__ pool, uint32_t* err)
 {
     constexpr int L = (1 << (BITS - 1)) - 1;
     constexpr int CB = kHeadDim * BITS / 8;   // code bytes per row
@@ -184,7 +184,8 @@ k_quantize_append(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v
         u[e] = (uint32_t)(code + L);
     }
 
-    uint8_t* blk = (which ? vp : kp) + (page * num_kv_heads + head) * block_bytes;
+    // pool[page][head][K block, V block]
+    uint8_t* blk = pool + ((page * num_kv_heads + head) * 2 + which) * block_bytes;
     if (!which) {
         // K: the packed vector is token row `off`
         store_codes<BITS>(blk + (int64_t)off * CB, u, lane, k_swizzle<BITS>(off));
@@ -199,8 +200,7 @@ k_quantize_append(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v
 __global__ void __launch_bounds__(32 * kAppendWarps)
 k_append_bf16(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
               const int64_t* __restrict__ slots, int num_tokens, int num_kv_heads,
-              int page_size, int num_pages, uint16_t* __restrict__ kp,
-              uint16_t* __restrict__ vp, uint32_t* err)
+              int page_size, int num_pages, uint16_t* __restrict__ pool, uint32_t* err)
 {
     const int lane = threadIdx.x & 31;
     const int64_t vec = (int64_t)blockIdx.x * kAppendWarps + (threadIdx.x >> 5);
@@ -219,8 +219,8 @@ k_append_bf16(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
         return;
     }
     const uint16_t* src = (which ? v : k) + (tok * num_kv_heads + head) * kHeadDim;
-    uint16_t* dst = (which ? vp : kp) +
-                    ((page * num_kv_heads + head) * page_size + off) * kHeadDim;
+    uint16_t* dst = pool + ((((page * num_kv_heads + head) * 2 + which) * page_size + off) *
+                            kHeadDim);
     reinterpret_cast<uint2*>(dst)[lane] = __ldg(reinterpret_cast<const uint2*>(src) + lane);
 }
 
@@ -234,12 +234,11 @@ cudaError_t launch_quantize_append(const void* k, const void* v, const int64_t* 
     const unsigned grid = (unsigned)((vecs + kAppendWarps - 1) / kAppendWarps);
     const auto* kk = static_cast<const uint16_t*>(k);
     const auto* vv = static_cast<const uint16_t*>(v);
-    auto* kp = static_cast<uint8_t*>(c.k_pages);
-    auto* vp = static_cast<uint8_t*>(c.v_pages);
+    auto* pool = static_cast<uint8_t*>(c.pages);
 #define TQ_LAUNCH_QA(B)                                                               \
     k_quantize_append<B><<<grid, 32 * kAppendWarps, 0, stream>>>(                     \
         kk, vv, slots, num_tokens, c.num_kv_heads, c.page_size, c.num_pages,         \
-        block_bytes, kp, vp, c.dev_error)
+        block_bytes, pool, c.dev_error)
     switch (bits) {
     case 2: TQ_LAUNCH_QA(2); break;
     case 3: TQ_LAUNCH_QA(3); break;
@@ -258,8 +257,7 @@ cudaError_t launch_append_bf16(const void* k, const void* v, const int64_t* slot
     const unsigned grid = (unsigned)((vecs + kAppendWarps - 1) / kAppendWarps);
     k_append_bf16<<<grid, 32 * kAppendWarps, 0, stream>>>(
         static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v), slots, num_tokens,
-        c.num_kv_heads, c.page_size, c.num_pages, static_cast<uint16_t*>(c.k_pages),
-        static_cast<uint16_t*>(c.v_pages), c.dev_error);
+        c.num_kv_heads, c.page_size, c.num_pages, static_cast<uint16_t*>(c.pages), c.dev_error);
     return cudaGetLastError();
 }
 

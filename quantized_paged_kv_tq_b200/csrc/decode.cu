@@ -1,9 +1,9 @@
-// Paged decode / speculative-verify attention over a TurboQuant or bf16 cache.
+// Paged decode / speculative-verify attention over the bf16 cache: the
+// uncompressed reference point beside the TurboQuant decode (decode_tc.cu),
+// and the split-size / workspace bookkeeping both decodes share.
 //
-// "xInfer: Pure-Rust LLM Inference Without a Python Runtime", section
-// "TurboQuant is a memory trade": reading a low-bit KV cache dequantises on
-// every attention step.  "infero", section "Continuous batching": a running
-// batch shares the GPU over a paged KV cache.
+// "infero", section "Continuous batching": a running batch shares the GPU
+// over a paged KV cache.
 //
 // Work decomposition (split-KV):
 //   grid = (max splits, kv heads x row groups, batch), 4 warps per CTA.
@@ -13,22 +13,20 @@
 //   of the kv head (up to 8 per row group) share every byte read.
 //   Each warp streams its own 16-token tiles (tile w, w+4, ...) through a
 //   private ring of shared-memory stages filled by 1-D bulk async copies
-//   (cp.async.bulk + mbarrier; codes and fp32 scales of K and V).
+//   (cp.async.bulk + mbarrier) of the K and V rows.
 //
 // Per tile (16 tokens):
-//   QK^T  mma.sync m16n8k16, A = K codes unpacked in registers to exact f16
-//         integers (magic-number trick), B = the rotated query split into f16
-//         hi + lo parts (8 columns = 4 rows x {hi, lo}); fp32 accumulate.
-//         score = raw * (s_k / L) in log2 units.
+//   QK^T  mma.sync m16n8k16 with bf16 K rows as A and the query (scaled to
+//         log2 units, power-of-two prescale) split into bf16 hi + lo
+//         columns as B; fp32 accumulate.
 //   softmax online, with a lazy rescale: the running max only moves when a
 //         tile exceeds it by 2^8; causal limit j <= seq_len - q_len + t.
-//   PV    mma.sync with A = V codes (dims on M, tokens on K) and B = P' =
-//         p * s_v / L (hi + lo f16) transposed in registers by movmatrix.
-//         A running power-of-two V-scale exponent keeps P' inside f16 range.
+//   PV    mma.sync with A = V rows (dims on M, tokens on K) and B = P split
+//         into bf16 hi + lo, transposed in registers by movmatrix.
 // Epilogue: the 4 warps merge in shared memory; a sequence with one split
 // finishes directly, otherwise the CTA stores (m, l, O) partials and the last
 // CTA of the (sequence, kv head, row group), found with an atomic ticket,
-// merges all splits, rotates back (H o / sqrt(d)) and writes fp32 output.
+// merges all splits and writes fp32 output.
 #include <cstdint>
 #include <math_constants.h>
 
@@ -65,12 +63,10 @@ constexpr int kRowsPerCta = 8;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazyThreshold = 8.f;       // log2 units
 constexpr uint32_t kWaitSpins = 1u << 24;   // bounded mbarrier polls
-constexpr uint32_t kMagic = 0x64006400u;    // f16 pair (1024, 1024)
 
 struct DecodeArgs {
     const uint16_t* q;
-    const uint8_t* kp;
-    const uint8_t* vp;
+    const uint8_t* kv;         // pool[page][kv head][K block, V block]
     const int32_t* page_table;
     const int32_t* seq_lens;
     float* out;
@@ -94,14 +90,14 @@ struct DecodeArgs {
     int stages;
 };
 
+// Staging of the bf16 cache: 16 token rows of d bf16 values for K, then V.
 template <int BITS>
 struct Fmt {
-    static constexpr bool kTurbo = BITS != 16;
-    static constexpr int CB = kTurbo ? kHeadDim * BITS / 8 : 2 * kHeadDim;  // row bytes
+    static_assert(BITS == 16, "the mma.sync kernel serves the bf16 cache");
+    static constexpr int CB = 2 * kHeadDim;            // row bytes
     static constexpr int kTileCodes = 16 * CB;
-    static constexpr int kVOff = kTurbo ? kTileCodes + 64 : kTileCodes;
+    static constexpr int kVOff = kTileCodes;
     static constexpr int kStageBytes = 2 * kVOff;
-    static constexpr int L = kTurbo ? (1 << (BITS - 1)) - 1 : 1;
 };
 
 // QK^T tile row r (0..15) holds tile token perm(r); chosen so that the
@@ -117,83 +113,27 @@ __device__ __forceinline__ int perm(int r)
 template <int BITS>
 __device__ __forceinline__ int qk_dim(int t, int c, int f, int e)
 {
-    if constexpr (BITS == 4 || BITS == 3) return 32 * t + 8 * (c >> 1) + 2 * (c & 1) + f + 4 * e;
-    if constexpr (BITS == 8) return 32 * t + 4 * c + f + 2 * e;
-    if constexpr (BITS == 2) return 32 * t + 16 * (c >> 2) + 2 * (c & 3) + f + 8 * e;
-    return 32 * t + 8 * (c >> 1) + 4 * (c & 1) + 2 * f + e;  // bf16
+    return 32 * t + 8 * (c >> 1) + 4 * (c & 1) + 2 * f + e;
 }
 
-// ----------------------------------------------------------- K unpackers
-// ka[c][f]: f16x2 (bf16x2) A-fragment element pair for chunk c, half f, of
-// one token row; `row` points at that token's code bytes in the stage.
+// ----------------------------------------------------------- K rows
+// ka[c][f]: bf16x2 A-fragment element pair for chunk c, half f, of one token
+// row (dims 32t .. 32t + 31, adjacent pairs as stored); `row` points at that
+// token's row in the stage.
 template <int BITS>
 __device__ __forceinline__ void unpack_k(const uint8_t* row, int t, uint32_t ka[8][2])
 {
-    if constexpr (BITS == 4) {
-        const uint4 w = *reinterpret_cast<const uint4*>(row + 16 * t);
-        const uint32_t words[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-        for (int wi = 0; wi < 4; ++wi)
-#pragma unroll
-            for (int hb = 0; hb < 2; ++hb) {
-                const uint32_t x = hb ? words[wi] >> 8 : words[wi];
-                ka[2 * wi + hb][0] = hfma2_u32(and_or(x, 0x000F000Fu, kMagic), 0x3C003C00u, 0xE407E407u);
-                ka[2 * wi + hb][1] = hfma2_u32(and_or(x, 0x00F000F0u, kMagic), 0x2C002C00u, 0xD470D470u);
-            }
-    } else if constexpr (BITS == 8) {
-        const uint4 w0 = *reinterpret_cast<const uint4*>(row + 32 * t);
-        const uint4 w1 = *reinterpret_cast<const uint4*>(row + 32 * t + 16);
-        const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            ka[c][0] = hfma2_u32(prmt(words[c], 0x64646464u, 0x4240u), 0x3C003C00u, 0xE47FE47Fu);
-            ka[c][1] = hfma2_u32(prmt(words[c], 0x64646464u, 0x4341u), 0x3C003C00u, 0xE47FE47Fu);
-        }
-    } else if constexpr (BITS == 2) {
-        const uint2 w = *reinterpret_cast<const uint2*>(row + 8 * t);
-        const uint32_t words[2] = {w.x, w.y};
-        constexpr uint32_t mul[4] = {0x3C003C00u, 0x34003400u, 0x2C002C00u, 0x24002400u};
-        constexpr uint32_t add[4] = {0xE401E401u, 0xDC04DC04u, 0xD410D410u, 0xCC40CC40u};
-#pragma unroll
-        for (int wi = 0; wi < 2; ++wi)
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint32_t x = j < 4 ? words[wi] : words[wi] >> 8;
-                const int jj = j & 3;
-                ka[4 * wi + (j >> 1)][j & 1] =
-                    hfma2_u32(and_or(x, 0x00030003u << (2 * jj), kMagic), mul[jj], add[jj]);
-            }
-    } else if constexpr (BITS == 3) {
-        const uint32_t* p = reinterpret_cast<const uint32_t*>(row + 12 * t);
-        const uint32_t W0 = p[0], W1 = p[1], W2 = p[2];
-        const uint32_t G[4] = {W0, prmt(W0, W1, 0x6543u), prmt(W1, W2, 0x5432u), W2 >> 8};
-        constexpr uint32_t mul[3] = {0x3C003C00u, 0x30003000u, 0x24002400u};
-        constexpr uint32_t add[3] = {0xE403E403u, 0xD818D818u, 0xCCC0CCC0u};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint32_t sel = bitsel(G[q], G[q] << 4, 0x0000FFFFu);
-            const uint32_t sel3 = bitsel(G[q] >> 3, G[q] << 1, 0x0000FFFFu);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t pr = k < 3 ? and_or(sel, 0x00070007u << (3 * k), kMagic)
-                                          : and_or(sel3, 0x01C001C0u, kMagic);
-                const int kk = k < 3 ? k : 2;
-                ka[2 * q + (k >> 1)][k & 1] = hfma2_u32(pr, mul[kk], add[kk]);
-            }
-        }
-    } else {  // bf16: dims 32t .. 32t+31, adjacent pairs as stored
-#pragma unroll
-        for (int w4 = 0; w4 < 4; ++w4) {
-            const uint4 x = *reinterpret_cast<const uint4*>(row + 64 * t + 16 * w4);
-            ka[2 * w4][0] = x.x;
-            ka[2 * w4][1] = x.y;
-            ka[2 * w4 + 1][0] = x.z;
-            ka[2 * w4 + 1][1] = x.w;
-        }
+    for (int w4 = 0; w4 < 4; ++w4) {
+        const uint4 x = *reinterpret_cast<const uint4*>(row + 64 * t + 16 * w4);
+        ka[2 * w4][0] = x.x;
+        ka[2 * w4][1] = x.y;
+        ka[2 * w4 + 1][0] = x.z;
+        ka[2 * w4 + 1][1] = x.w;
     }
 }
 
-// ----------------------------------------------------------- V unpackers
+// ----------------------------------------------------------- V rows
 // va[mt][i]: A-fragment of V^T for m-tile mt (rows = dims 16g + 2mt and
 // 16g + 2mt + 1), k = tokens {t, t+4} (i = 0, 1) and {t+8, t+12} (i = 2, 3).
 template <int BITS>
@@ -204,131 +144,24 @@ __device__ __forceinline__ void unpack_v(const uint8_t* codes, int g, int t, uin
     const uint8_t* r1 = codes + (t + 4) * CB;
     const uint8_t* r2 = codes + (t + 8) * CB;
     const uint8_t* r3 = codes + (t + 12) * CB;
-    if constexpr (BITS == 4) {
-        const uint2 X[4] = {*reinterpret_cast<const uint2*>(r0 + 8 * g),
-                            *reinterpret_cast<const uint2*>(r1 + 8 * g),
-                            *reinterpret_cast<const uint2*>(r2 + 8 * g),
-                            *reinterpret_cast<const uint2*>(r3 + 8 * g)};
+    uint4 X[4][2];
+    const uint8_t* rows[4] = {r0, r1, r2, r3};
 #pragma unroll
-        for (int p = 0; p < 2; ++p)
+    for (int i = 0; i < 4; ++i) {
+        X[i][0] = *reinterpret_cast<const uint4*>(rows[i] + 32 * g);
+        X[i][1] = *reinterpret_cast<const uint4*>(rows[i] + 32 * g + 16);
+    }
 #pragma unroll
-            for (int hw = 0; hw < 2; ++hw) {
-                const uint32_t xw = hw ? X[2 * p].y : X[2 * p].x;
-                const uint32_t yw = hw ? X[2 * p + 1].y : X[2 * p + 1].x;
+    for (int p = 0; p < 2; ++p) {
+        const uint32_t xa[8] = {X[2 * p][0].x, X[2 * p][0].y, X[2 * p][0].z, X[2 * p][0].w,
+                                X[2 * p][1].x, X[2 * p][1].y, X[2 * p][1].z, X[2 * p][1].w};
+        const uint32_t ya[8] = {X[2 * p + 1][0].x, X[2 * p + 1][0].y, X[2 * p + 1][0].z,
+                                X[2 * p + 1][0].w, X[2 * p + 1][1].x, X[2 * p + 1][1].y,
+                                X[2 * p + 1][1].z, X[2 * p + 1][1].w};
 #pragma unroll
-                for (int xs = 0; xs < 2; ++xs) {
-                    const uint32_t xx = prmt(xw, yw, xs ? 0x7632u : 0x5410u);
-                    const uint32_t x8 = xx >> 8;
-                    const uint32_t d[4] = {
-                        hfma2_u32(and_or(xx, 0x000F000Fu, kMagic), 0x3C003C00u, 0xE407E407u),
-                        hfma2_u32(and_or(xx, 0x00F000F0u, kMagic), 0x2C002C00u, 0xD470D470u),
-                        hfma2_u32(and_or(x8, 0x000F000Fu, kMagic), 0x3C003C00u, 0xE407E407u),
-                        hfma2_u32(and_or(x8, 0x00F000F0u, kMagic), 0x2C002C00u, 0xD470D470u)};
-#pragma unroll
-                    for (int n = 0; n < 4; ++n) {
-                        const int dl = 8 * hw + 4 * xs + n;   // dim 16g + dl
-                        va[dl >> 1][(dl & 1) + 2 * p] = d[n];
-                    }
-                }
-            }
-    } else if constexpr (BITS == 8) {
-        const uint4 X[4] = {*reinterpret_cast<const uint4*>(r0 + 16 * g),
-                            *reinterpret_cast<const uint4*>(r1 + 16 * g),
-                            *reinterpret_cast<const uint4*>(r2 + 16 * g),
-                            *reinterpret_cast<const uint4*>(r3 + 16 * g)};
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            const uint32_t xa[4] = {X[2 * p].x, X[2 * p].y, X[2 * p].z, X[2 * p].w};
-            const uint32_t ya[4] = {X[2 * p + 1].x, X[2 * p + 1].y, X[2 * p + 1].z, X[2 * p + 1].w};
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const uint32_t t1 = prmt(xa[w], ya[w], 0x5410u);
-                const uint32_t t2 = prmt(xa[w], ya[w], 0x7632u);
-                const uint32_t d[4] = {
-                    hfma2_u32(prmt(t1, 0x64646464u, 0x4240u), 0x3C003C00u, 0xE47FE47Fu),
-                    hfma2_u32(prmt(t1, 0x64646464u, 0x4341u), 0x3C003C00u, 0xE47FE47Fu),
-                    hfma2_u32(prmt(t2, 0x64646464u, 0x4240u), 0x3C003C00u, 0xE47FE47Fu),
-                    hfma2_u32(prmt(t2, 0x64646464u, 0x4341u), 0x3C003C00u, 0xE47FE47Fu)};
-#pragma unroll
-                for (int n = 0; n < 4; ++n) {
-                    const int dl = 4 * w + n;
-                    va[dl >> 1][(dl & 1) + 2 * p] = d[n];
-                }
-            }
-        }
-    } else if constexpr (BITS == 2) {
-        const uint32_t X[4] = {*reinterpret_cast<const uint32_t*>(r0 + 4 * g),
-                               *reinterpret_cast<const uint32_t*>(r1 + 4 * g),
-                               *reinterpret_cast<const uint32_t*>(r2 + 4 * g),
-                               *reinterpret_cast<const uint32_t*>(r3 + 4 * g)};
-        constexpr uint32_t mul[4] = {0x3C003C00u, 0x34003400u, 0x2C002C00u, 0x24002400u};
-        constexpr uint32_t add[4] = {0xE401E401u, 0xDC04DC04u, 0xD410D410u, 0xCC40CC40u};
-#pragma unroll
-        for (int p = 0; p < 2; ++p)
-#pragma unroll
-            for (int xi = 0; xi < 2; ++xi) {
-                const uint32_t xx = prmt(X[2 * p], X[2 * p + 1], xi ? 0x7632u : 0x5410u);
-                const uint32_t x8 = xx >> 8;
-#pragma unroll
-                for (int n = 0; n < 8; ++n) {
-                    const int jj = n & 3;
-                    const uint32_t v = hfma2_u32(
-                        and_or(n < 4 ? xx : x8, 0x00030003u << (2 * jj), kMagic), mul[jj], add[jj]);
-                    const int dl = 8 * xi + n;
-                    va[dl >> 1][(dl & 1) + 2 * p] = v;
-                }
-            }
-    } else if constexpr (BITS == 3) {
-        // 48 bits per token at bit 48g; read two aligned words and shift
-        const int byte0 = 6 * g;
-        const int base = byte0 & ~3;
-        const int sh = (byte0 & 3) * 8;
-        uint64_t bits[4];
-        const uint8_t* rows[4] = {r0, r1, r2, r3};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t* w = reinterpret_cast<const uint32_t*>(rows[i] + base);
-            const uint64_t v64 = ((uint64_t)w[1] << 32) | w[0];
-            bits[i] = v64 >> sh;
-        }
-        constexpr uint32_t mul[3] = {0x3C003C00u, 0x30003000u, 0x24002400u};
-        constexpr uint32_t add[3] = {0xE403E403u, 0xD818D818u, 0xCCC0CCC0u};
-#pragma unroll
-        for (int p = 0; p < 2; ++p)
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const uint32_t a12 = (uint32_t)(bits[2 * p] >> (12 * m)) & 0xFFFu;
-                const uint32_t b12 = (uint32_t)(bits[2 * p + 1] >> (12 * m)) & 0xFFFu;
-                const uint32_t xy = a12 | (b12 << 16);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint32_t pr = k < 3 ? and_or(xy, 0x00070007u << (3 * k), kMagic)
-                                              : and_or(xy >> 3, 0x01C001C0u, kMagic);
-                    const int kk = k < 3 ? k : 2;
-                    const int dl = 4 * m + k;
-                    va[dl >> 1][(dl & 1) + 2 * p] = hfma2_u32(pr, mul[kk], add[kk]);
-                }
-            }
-    } else {  // bf16
-        uint4 X[4][2];
-        const uint8_t* rows[4] = {r0, r1, r2, r3};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            X[i][0] = *reinterpret_cast<const uint4*>(rows[i] + 32 * g);
-            X[i][1] = *reinterpret_cast<const uint4*>(rows[i] + 32 * g + 16);
-        }
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            const uint32_t xa[8] = {X[2 * p][0].x, X[2 * p][0].y, X[2 * p][0].z, X[2 * p][0].w,
-                                    X[2 * p][1].x, X[2 * p][1].y, X[2 * p][1].z, X[2 * p][1].w};
-            const uint32_t ya[8] = {X[2 * p + 1][0].x, X[2 * p + 1][0].y, X[2 * p + 1][0].z,
-                                    X[2 * p + 1][0].w, X[2 * p + 1][1].x, X[2 * p + 1][1].y,
-                                    X[2 * p + 1][1].z, X[2 * p + 1][1].w};
-#pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
-                va[mt][2 * p] = prmt(xa[mt], ya[mt], 0x5410u);
-                va[mt][2 * p + 1] = prmt(xa[mt], ya[mt], 0x7632u);
-            }
+        for (int mt = 0; mt < 8; ++mt) {
+            va[mt][2 * p] = prmt(xa[mt], ya[mt], 0x5410u);
+            va[mt][2 * p + 1] = prmt(xa[mt], ya[mt], 0x7632u);
         }
     }
 }
@@ -338,23 +171,18 @@ __device__ __forceinline__ void issue_tile(uint8_t* dst, uint64_t* bar, const De
                                            int page, int kvh, int sub, bool one_block)
 {
     using F = Fmt<BITS>;
-    const int64_t blk = ((int64_t)page * a.num_kv_heads + kvh) * a.block_bytes;
-    const uint8_t* kb = a.kp + blk;
-    const uint8_t* vb = a.vp + blk;
+    const int64_t blk = ((int64_t)page * a.num_kv_heads + kvh) * 2 * a.block_bytes;
+    const uint8_t* kb = a.kv + blk;
+    const uint8_t* vb = kb + a.block_bytes;
     mbar_arrive_expect_tx(bar, F::kStageBytes);
     if (one_block) {
-        // a 16-token page is exactly one tile: codes then scales, as staged
+        // a 16-token page is exactly one tile
         bulk_g2s(dst, kb, F::kVOff, bar);
         bulk_g2s(dst + F::kVOff, vb, F::kVOff, bar);
         return;
     }
     bulk_g2s(dst, kb + sub * F::kTileCodes, F::kTileCodes, bar);
     bulk_g2s(dst + F::kVOff, vb + sub * F::kTileCodes, F::kTileCodes, bar);
-    if constexpr (F::kTurbo) {
-        const int64_t so = (int64_t)a.page_size * F::CB + 64 * sub;
-        bulk_g2s(dst + F::kTileCodes, kb + so, 64, bar);
-        bulk_g2s(dst + F::kVOff + F::kTileCodes, vb + so, 64, bar);
-    }
 }
 
 template <int BITS, int NT>
@@ -434,13 +262,7 @@ k_decode(const DecodeArgs a)
             x[2] = bf16_bits_to_float(raw.y & 0xffffu);
             x[3] = bf16_bits_to_float(raw.y >> 16);
         }
-        float fac;
-        if constexpr (F::kTurbo) {
-            fwht128_lane(x, lane);
-            fac = kLog2e / kHeadDim;        // (H q / sqrt d) . y / sqrt d = (H q) . y / d
-        } else {
-            fac = kLog2e * 0.08838834764831845f;  // 1 / sqrt(128)
-        }
+        const float fac = kLog2e * 0.08838834764831845f;  // 1 / sqrt(128)
         float amax = 0.f;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -473,15 +295,9 @@ k_decode(const DecodeArgs a)
             for (int f = 0; f < 2; ++f) {
                 const float v0 = qrow[qk_dim<BITS>(t, c, f, 0)];
                 const float v1 = qrow[qk_dim<BITS>(t, c, f, 1)];
-                if constexpr (F::kTurbo) {
-                    const float h0 = __half2float(__float2half_rn(v0));
-                    const float h1 = __half2float(__float2half_rn(v1));
-                    qf[nt][c][f] = g < 4 ? pack_half2(v0, v1) : pack_half2(v0 - h0, v1 - h1);
-                } else {
-                    const float h0 = __bfloat162float(__float2bfloat16_rn(v0));
-                    const float h1 = __bfloat162float(__float2bfloat16_rn(v1));
-                    qf[nt][c][f] = g < 4 ? pack_bf162(v0, v1) : pack_bf162(v0 - h0, v1 - h1);
-                }
+                const float h0 = __bfloat162float(__float2bfloat16_rn(v0));
+                const float h1 = __bfloat162float(__float2bfloat16_rn(v1));
+                qf[nt][c][f] = g < 4 ? pack_bf162(v0, v1) : pack_bf162(v0 - h0, v1 - h1);
             }
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
@@ -506,12 +322,6 @@ k_decode(const DecodeArgs a)
             l_run[nt][e] = 0.f;
         }
     }
-    // V scales: P' = p * s_v / L * 2^(127 - ev) with ev the largest biased
-    // fp32 exponent of the scales seen so far, so P' stays below 2^9 in f16
-    int ev = 0;
-    float vn = 1.f;                              // 2^(127 - ev)
-    float vlimit = __uint_as_float(1u << 23);    // scales >= this raise ev
-    const float kinv = F::kTurbo ? 1.f / (float)F::L : 1.f;
     const int ra = perm(g), rb = perm(g + 8);
     // a tile is fully visible when its last token is within the causal limit
     // of the first (most restricted) row of this row group
@@ -547,8 +357,7 @@ k_decode(const DecodeArgs a)
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     float* acc = c < 4 ? s[nt] : s2[nt];
-                    if constexpr (F::kTurbo) mma_f16(acc, afr, qf[nt][c][0], qf[nt][c][1]);
-                    else mma_bf16(acc, afr, qf[nt][c][0], qf[nt][c][1]);
+                    mma_bf16(acc, afr, qf[nt][c][0], qf[nt][c][1]);
                 }
             }
             // hi + lo columns (lanes t and t ^ 2)
@@ -560,20 +369,13 @@ k_decode(const DecodeArgs a)
                     s[nt][k] += __shfl_xor_sync(kFull, s[nt][k], 2);
                 }
         }
-        float ks0 = kinv, ks1 = kinv, vs0 = 1.f, vs1 = 1.f;
-        if constexpr (F::kTurbo) {
-            const float* kscale = reinterpret_cast<const float*>(st + F::kTileCodes);
-            const float* vscale = reinterpret_cast<const float*>(st + F::kVOff + F::kTileCodes);
-            ks0 = kscale[ra] * kinv;
-            ks1 = kscale[rb] * kinv;
-            vs0 = vscale[ra] * kinv;
-            vs1 = vscale[rb] * kinv;
-        }
+        // 1 for a token of the sequence, 0 for a slot past its end
+        float ks0 = 1.f, ks1 = 1.f, vs0 = 1.f, vs1 = 1.f;
         const bool full = tok0 + 15 <= lim_min;     // warp-uniform
         const int ja = tok0 + ra, jb = tok0 + rb;
         if (!full) {
-            // slots past the sequence end were never written: keep their
-            // (arbitrary) scales out of every product
+            // slots past the sequence end were never written: keep them out
+            // of every product
             if (ja >= seq_len) { ks0 = 0.f; vs0 = 0.f; }
             if (jb >= seq_len) { ks1 = 0.f; vs1 = 0.f; }
         }
@@ -594,18 +396,7 @@ k_decode(const DecodeArgs a)
                 sc[nt][2 + e] = x1;
                 need |= fmaxf(x0, x1) > m_run[nt][e] + kLazyThreshold;
             }
-        if constexpr (F::kTurbo) need |= fmaxf(vs0, vs1) >= vlimit;
         if (__any_sync(kFull, need)) {
-            float av = 1.f;
-            if constexpr (F::kTurbo) {
-                // non-negative floats order like their bit patterns
-                const unsigned vb = __reduce_max_sync(kFull, __float_as_uint(fmaxf(vs0, vs1)));
-                const int ev_new = max(ev, (int)(vb >> 23));
-                av = pow2i(ev - ev_new);
-                ev = ev_new;
-                vn = pow2i(127 - ev);
-                vlimit = ev >= 254 ? CUDART_INF_F : __uint_as_float((uint32_t)(ev + 1) << 23);
-            }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -618,17 +409,16 @@ k_decode(const DecodeArgs a)
                     const float alpha = mn == -CUDART_INF_F ? 1.f : fast_exp2(m_run[nt][e] - mn);
                     m_run[nt][e] = mn;
                     l_run[nt][e] *= alpha;
-                    const float ao = alpha * av;
 #pragma unroll
                     for (int mt = 0; mt < 8; ++mt) {
-                        o[nt][mt][e] *= ao;
-                        o[nt][mt][2 + e] *= ao;
+                        o[nt][mt][e] *= alpha;
+                        o[nt][mt][2 + e] *= alpha;
                     }
                 }
         }
-        // P' = p * s_v / L * 2^(127 - ev), split into hi (lanes t < 2) and
-        // lo (t >= 2) halves, transposed onto the PV B fragment
-        const float vn0 = vs0 * vn, vn1 = vs1 * vn;
+        // P, split into hi (lanes t < 2) and lo (t >= 2) bf16 halves,
+        // transposed onto the PV B fragment
+        const float vn0 = vs0, vn1 = vs1;
         uint32_t pb[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -646,14 +436,13 @@ k_decode(const DecodeArgs a)
                 pv[e] = p0 * vn0;
                 pv[2 + e] = p1 * vn1;
                 if (!full) {
-                    // a masked token may carry a scale above the running
-                    // exponent: 0 * (overflowed scale) must stay 0
+                    // a masked entry stays exactly 0
                     pv[e] = p0 > 0.f ? pv[e] : 0.f;
                     pv[2 + e] = p1 > 0.f ? pv[2 + e] : 0.f;
                 }
             }
-            pb[nt][0] = movmatrix_trans(split_hi_lo<F::kTurbo>(pv[0], pv[1], t < 2));
-            pb[nt][1] = movmatrix_trans(split_hi_lo<F::kTurbo>(pv[2], pv[3], t < 2));
+            pb[nt][0] = movmatrix_trans(split_hi_lo<false>(pv[0], pv[1], t < 2));
+            pb[nt][1] = movmatrix_trans(split_hi_lo<false>(pv[2], pv[3], t < 2));
         }
 
         // ---------------- O^T += V^T P'
@@ -664,8 +453,7 @@ k_decode(const DecodeArgs a)
             for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    if constexpr (F::kTurbo) mma_f16(o[nt][mt], va[mt], pb[nt][0], pb[nt][1]);
-                    else mma_bf16(o[nt][mt], va[mt], pb[nt][0], pb[nt][1]);
+                    mma_bf16(o[nt][mt], va[mt], pb[nt][0], pb[nt][1]);
                 }
         }
 
@@ -702,14 +490,13 @@ k_decode(const DecodeArgs a)
             l += __shfl_xor_sync(kFull, l, 16);
             l_run[nt][e] = l;
         }
-    const float vback = F::kTurbo ? pow2i(ev - 127) : 1.f;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                o[nt][mt][i] = (o[nt][mt][i] + __shfl_xor_sync(kFull, o[nt][mt][i], 2)) * vback;
+                o[nt][mt][i] = o[nt][mt][i] + __shfl_xor_sync(kFull, o[nt][mt][i], 2);
 
     __syncthreads();  // every warp is done with its ring
     float* sO = reinterpret_cast<float*>(ring);                          // [4][8][128]
@@ -740,7 +527,6 @@ k_decode(const DecodeArgs a)
     const int nrows = min(kRowsPerCta, min(4 * NT, a.G - rg * kRowsPerCta));
     const int64_t unit = ((int64_t)b * gridDim.y + blockIdx.y);        // (seq, kvh, rg)
     const int64_t part = unit * a.max_splits + split;
-    const float rs = 0.08838834764831845f;                             // 1 / sqrt(128)
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
         const int rr = warp + 4 * k;
@@ -768,11 +554,6 @@ k_decode(const DecodeArgs a)
         if (nsplit == 1) {
             const float inv = 1.f / Lsum;
             float x[4] = {acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv};
-            if constexpr (F::kTurbo) {
-                fwht128_lane(x, lane);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) x[e] *= rs;
-            }
             *reinterpret_cast<float4*>(a.out + (((int64_t)b * a.q_len + tq) * a.num_q_heads + h) *
                                                    kHeadDim + 4 * lane) =
                 make_float4(x[0], x[1], x[2], x[3]);
@@ -816,11 +597,6 @@ k_decode(const DecodeArgs a)
         }
         const float inv = 1.f / Lsum;
         float x[4] = {acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv};
-        if constexpr (F::kTurbo) {
-            fwht128_lane(x, lane);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) x[e] *= rs;
-        }
         const int r = rg * kRowsPerCta + rr;
         const int tq = r / a.group;
         const int h = kvh * a.group + (r - tq * a.group);
@@ -878,8 +654,8 @@ cudaError_t launch_decode_tc(const void* q, const tq_cache& c, int64_t block_byt
                              int batch, int q_len, int num_q_heads, int max_seq_len, float* out,
                              void* workspace, int split_tokens, cudaStream_t stream);
 
-// Query rows per CTA: the tensor-core kernel (turbo formats) takes 8 or 16,
-// the warp-MMA kernel (bf16) 8.
+// Query rows per CTA: the tensor-core kernels (turbo formats) take 4, 8 or
+// 16 (decode_tc_rows), the warp-MMA kernel (bf16) 8.
 int decode_rows_per_cta(int format, int G)
 {
     return format == 16 ? kRowsPerCta : decode_tc_rows(format, G);
@@ -917,8 +693,7 @@ cudaError_t launch_decode(const void* q, const tq_cache& c, int64_t block_bytes,
                                 decode_split_tokens(c.page_size), stream);
     DecodeArgs a{};
     a.q = static_cast<const uint16_t*>(q);
-    a.kp = static_cast<const uint8_t*>(c.k_pages);
-    a.vp = static_cast<const uint8_t*>(c.v_pages);
+    a.kv = static_cast<const uint8_t*>(c.pages);
     a.page_table = page_table;
     a.seq_lens = seq_lens;
     a.out = out;

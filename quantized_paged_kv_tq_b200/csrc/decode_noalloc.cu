@@ -87,8 +87,8 @@ TQ_API tq_status tq_paged_decode_noalloc(const void* q, const tq_cache* cache,
     if (cache->head_dim != 128) return TQ_ERR_UNSUPPORTED;
     if (cache->page_size != 16 && cache->page_size != 32 && cache->page_size != 64)
         return TQ_ERR_UNSUPPORTED;
-    if (!cache->k_pages || !cache->v_pages || !aligned16(cache->k_pages) ||
-        !aligned16(cache->v_pages) || (reinterpret_cast<uintptr_t>(cache->dev_error) & 3u))
+    if (!cache->pages || !aligned16(cache->pages) ||
+        (reinterpret_cast<uintptr_t>(cache->dev_error) & 3u))
         return TQ_ERR_INVALID_ARG;
     if (batch < 0 || q_len <= 0 || num_q_heads <= 0 || max_seq_len <= 0) return TQ_ERR_INVALID_ARG;
     if (num_q_heads % cache->num_kv_heads || max_seq_len < q_len) return TQ_ERR_INVALID_ARG;

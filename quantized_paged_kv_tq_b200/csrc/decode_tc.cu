@@ -46,8 +46,7 @@ constexpr uint32_t kMagicTc = 0x64006400u;
 
 struct TcArgs {
     const uint16_t* q;
-    const uint8_t* kp;
-    const uint8_t* vp;
+    const uint8_t* kv;         // pool[page][kv head][K block, V block]
     const int32_t* page_table;
     const int32_t* seq_lens;
     float* out;
@@ -192,8 +191,8 @@ __device__ __forceinline__ void k_row_to_tmem(const uint8_t* row, uint32_t taddr
 }
 
 // V codes of dimension `dim` for the 128 tokens of a tile -> tensor memory
-// columns [0, 64) of this thread's lane.  vblk0: first V block of the tile in
-// the stage; pages of P tokens follow each other every block_bytes.
+// columns [0, 64) of this thread's lane.  vblk0: V block of the tile's first
+// page in the stage; the V blocks of later pages follow every `bb` bytes.
 template <int BITS>
 __device__ __forceinline__ void v_col_to_tmem(const uint8_t* vblk0, int64_t bb, int lp, int dim,
                                               uint32_t taddr)
@@ -264,13 +263,13 @@ __device__ __forceinline__ void v_col_to_tmem(const uint8_t* vblk0, int64_t bb, 
     }
 }
 
-// Bulk copies of one tile's K and V page blocks into a stage (warp 0).
+// Bulk copies of one tile's pages into a stage (warp 0): one copy per page of
+// its adjacent K and V blocks, so the stage is [page][K block, V block].
 // pids[j]: physical page of the tile's j-th page (global page table or the
 // split's copy in shared memory).
 __device__ __forceinline__ void issue_tile_tc(uint8_t* stage, uint64_t* bar, const TcArgs& a,
                                               const int* pids, int kvh, int ntok, int lane)
 {
-    const int npp = kTile >> a.lp;                        // page slots per stage
     const int npg = (ntok + (1 << a.lp) - 1) >> a.lp;     // pages holding tokens
     if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(2 * npg * a.block_bytes));
     __syncwarp();
@@ -280,9 +279,8 @@ __device__ __forceinline__ void issue_tile_tc(uint8_t* stage, uint64_t* bar, con
             report_error(a.err, TQ_ERR_DEVICE_CHECK, kErrPageRange);
             pid = 0;
         }
-        const int64_t off = ((int64_t)pid * a.num_kv_heads + kvh) * a.block_bytes;
-        bulk_g2s(stage + lane * a.block_bytes, a.kp + off, (uint32_t)a.block_bytes, bar);
-        bulk_g2s(stage + (npp + lane) * a.block_bytes, a.vp + off, (uint32_t)a.block_bytes, bar);
+        const int64_t off = ((int64_t)pid * a.num_kv_heads + kvh) * 2 * a.block_bytes;
+        bulk_g2s(stage + lane * 2 * a.block_bytes, a.kv + off, (uint32_t)(2 * a.block_bytes), bar);
     }
 }
 
@@ -293,7 +291,6 @@ __device__ __forceinline__ void issue_tile_warps(uint8_t* stage, uint64_t* bar, 
                                                  const int* pids, int kvh, int ntok, int warp,
                                                  int lane)
 {
-    const int npp = kTile >> a.lp;
     const int npg = (ntok + (1 << a.lp) - 1) >> a.lp;
     const int mine = npg > warp ? (npg - warp + 3) >> 2 : 0;      // pages of this warp
     if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(2 * mine * a.block_bytes));
@@ -305,9 +302,8 @@ __device__ __forceinline__ void issue_tile_warps(uint8_t* stage, uint64_t* bar, 
             report_error(a.err, TQ_ERR_DEVICE_CHECK, kErrPageRange);
             pid = 0;
         }
-        const int64_t off = ((int64_t)pid * a.num_kv_heads + kvh) * a.block_bytes;
-        bulk_g2s(stage + j * a.block_bytes, a.kp + off, (uint32_t)a.block_bytes, bar);
-        bulk_g2s(stage + (npp + j) * a.block_bytes, a.vp + off, (uint32_t)a.block_bytes, bar);
+        const int64_t off = ((int64_t)pid * a.num_kv_heads + kvh) * 2 * a.block_bytes;
+        bulk_g2s(stage + j * 2 * a.block_bytes, a.kv + off, (uint32_t)(2 * a.block_bytes), bar);
     }
 }
 
@@ -446,7 +442,6 @@ k_decode_tc(const TcArgs a)
     const int tok_end = min(seq_len, tok_begin + a.split_tokens);
     const int ntiles = (tok_end - tok_begin + kTile - 1) / kTile;
     const int P = a.page_size;
-    const int npp = kTile >> a.lp;
 
     // ---- set-up: barriers, tensor memory, first copies
     if (tid == 0) {
@@ -570,8 +565,8 @@ k_decode_tc(const TcArgs a)
 
         // 1. K row of token tid -> A operand
         const int pg = tid >> a.lp, row = tid & (P - 1);
-        const uint8_t* kblk = st + pg * a.block_bytes;
-        const uint8_t* vblk = st + (npp + pg) * a.block_bytes;
+        const uint8_t* kblk = st + pg * 2 * a.block_bytes;     // stage: [page][K block, V block]
+        const uint8_t* vblk = kblk + a.block_bytes;
         k_row_to_tmem<BITS>(kblk + row * F::CB, t_lane);
         float ks = reinterpret_cast<const float*>(kblk + P * F::CB)[row] * kinv;
         float vs = reinterpret_cast<const float*>(vblk + P * F::CB)[row] * kinv;
@@ -599,7 +594,7 @@ k_decode_tc(const TcArgs a)
         uint32_t sraw[NCOL];
 #pragma unroll
         for (int c = 0; c < NCOL; c += 16) tmem_ld16(t_lane + kColS + c, sraw + c);
-        v_col_to_tmem<BITS>(st + npp * a.block_bytes, a.block_bytes, a.lp, tid, t_lane);
+        v_col_to_tmem<BITS>(st + a.block_bytes, 2 * a.block_bytes, a.lp, tid, t_lane);
         tmem_wait_ld();
         const bool full_tile = tok0 + kTile - 1 <= lim_min;
         float sc[RG];
@@ -867,7 +862,7 @@ __device__ __forceinline__ void k_row_to_tmem_u8(const uint8_t* row, uint32_t ta
 
 // V codes of dimension `dim` for the tile's 128 tokens -> 32 words of
 // unsigned bytes in K-position order (registers; stored once the previous
-// PV product has drained).
+// PV product has drained).  vblk0 and bb as for v_col_to_tmem.
 template <int BITS>
 __device__ __forceinline__ void v_col_u8(const uint8_t* vblk0, int64_t bb, int lp, int dim,
                                          uint32_t* o)
@@ -997,7 +992,6 @@ k_decode_i8(const TcArgs a)
     const int tok_end = min(seq_len, tok_begin + a.split_tokens);
     const int ntiles = (tok_end - tok_begin + kTile - 1) / kTile;
     const int P = a.page_size;
-    const int npp = kTile >> a.lp;
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) mbar_init(&full[s], kTcThreads / 32);
@@ -1167,8 +1161,8 @@ k_decode_i8(const TcArgs a)
     auto stage_k = [&](int t, float& ks_out, float& vs_out) {
         const uint8_t* st = ring + (t % kStages) * F::kStage;
         const int pg = tid >> a.lp, row = tid & (P - 1);
-        const uint8_t* kblk = st + pg * a.block_bytes;
-        const uint8_t* vblk = st + (npp + pg) * a.block_bytes;
+        const uint8_t* kblk = st + pg * 2 * a.block_bytes;     // stage: [page][K block, V block]
+        const uint8_t* vblk = kblk + a.block_bytes;
         k_row_to_tmem_u8<BITS>(kblk + row * F::CB, t_lane + kColAK, k_swizzle<BITS>(row));
         if constexpr (RG <= 4) {
             tmem_st16(t_lane + kColS, sinit);
@@ -1246,7 +1240,7 @@ k_decode_i8(const TcArgs a)
         // b. V column of dimension tid (registers), overlapping the load of
         // S for 4 rows; after the scores for 8 (register pressure)
         uint32_t vw[32];
-        if constexpr (RG <= 4) v_col_u8<BITS>(st + npp * a.block_bytes, a.block_bytes, a.lp, tid, vw);
+        if constexpr (RG <= 4) v_col_u8<BITS>(st + a.block_bytes, 2 * a.block_bytes, a.lp, tid, vw);
         tmem_wait_ld();
 
         const bool full_tile = tok0 + kTile - 1 <= lim_min;
@@ -1268,7 +1262,7 @@ k_decode_i8(const TcArgs a)
         }
         need |= vs >= vlimit;
         const float vs_t = vs;
-        if constexpr (RG > 4) v_col_u8<BITS>(st + npp * a.block_bytes, a.block_bytes, a.lp, tid, vw);
+        if constexpr (RG > 4) v_col_u8<BITS>(st + a.block_bytes, 2 * a.block_bytes, a.lp, tid, vw);
 
         // c. K codes of tile tt + 1 (S of tile tt is in registers)
         if (tt + 1 < ntiles) {
@@ -1448,8 +1442,7 @@ cudaError_t launch_decode_tc(const void* q, const tq_cache& c, int64_t block_byt
 {
     TcArgs a{};
     a.q = static_cast<const uint16_t*>(q);
-    a.kp = static_cast<const uint8_t*>(c.k_pages);
-    a.vp = static_cast<const uint8_t*>(c.v_pages);
+    a.kv = static_cast<const uint8_t*>(c.pages);
     a.page_table = page_table;
     a.seq_lens = seq_lens;
     a.out = out;

@@ -44,8 +44,8 @@ SYMBOLS = ("tq_abi_version", "tq_status_string", "tq_page_block_bytes",
 class tq_cache(ctypes.Structure):
     _fields_ = [("format", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("page_size", ctypes.c_int32),
-                ("num_pages", ctypes.c_int32), ("k_pages", ctypes.c_void_p),
-                ("v_pages", ctypes.c_void_p), ("dev_error", ctypes.c_void_p)]
+                ("num_pages", ctypes.c_int32), ("pages", ctypes.c_void_p),
+                ("dev_error", ctypes.c_void_p)]
 
 
 _P = ctypes.c_void_p
@@ -125,10 +125,12 @@ def tq_page_block_bytes(fmt: int, head_dim: int = 128, page_size: int = 16) -> i
 
 
 class Cache:
-    """Paged K/V pools of one layer plus its C descriptor.
+    """Paged K/V pool of one layer plus its C descriptor.
 
-    Pools are torch uint8 tensors [num_pages][num_kv_heads][block] (zeroed);
-    ``dev_error`` is a one-word int32 tensor the kernels report to.
+    ``pages`` is a zeroed torch uint8 tensor [num_pages][num_kv_heads][2][block]
+    (the K block, then the V block); ``k_pages`` and ``v_pages`` are its
+    [num_pages][num_kv_heads][block] views.  ``dev_error`` is a one-word int32 tensor
+    the kernels report to.
     """
 
     def __init__(self, fmt: int, num_pages: int, num_kv_heads: int, page_size: int = 16,
@@ -138,12 +140,14 @@ class Cache:
             raise ValueError("unsupported cache shape")
         self.format, self.num_pages, self.num_kv_heads = fmt, num_pages, num_kv_heads
         self.page_size, self.head_dim, self.block_bytes = page_size, head_dim, bb
-        self.k_pages = torch.zeros((num_pages, num_kv_heads, bb), dtype=torch.uint8, device=device)
-        self.v_pages = torch.zeros_like(self.k_pages)
+        # one pool [page][kv head][K block, V block]; k_pages / v_pages are views
+        self.pages = torch.zeros((num_pages, num_kv_heads, 2, bb), dtype=torch.uint8,
+                                 device=device)
+        self.k_pages = self.pages[:, :, 0]
+        self.v_pages = self.pages[:, :, 1]
         self.dev_error = torch.zeros(1, dtype=torch.int32, device=device)
         self.desc = tq_cache(fmt, head_dim, num_kv_heads, page_size, num_pages,
-                             self.k_pages.data_ptr(), self.v_pages.data_ptr(),
-                             self.dev_error.data_ptr())
+                             self.pages.data_ptr(), self.dev_error.data_ptr())
         self._ws = None
 
     def workspace(self, batch: int, q_len: int, num_q_heads: int, max_seq_len: int,

@@ -33,7 +33,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_strings():
-    assert tq.abi_version() == 1
+    assert tq.abi_version() == 2
     for s in range(7):
         assert tq.status_string(s).startswith("TQ_")
     assert tq.status_string(99) == "TQ_ERR_UNKNOWN"
@@ -57,8 +57,8 @@ def test_block_bytes():
 FAKE = 0x10000  # never dereferenced: every call below stops in host checks
 
 
-def desc(fmt=4, d=128, H=8, P=16, pages=10, kp=FAKE, vp=FAKE, err=None):
-    return tq.tq_cache(fmt, d, H, P, pages, kp, vp, err)
+def desc(fmt=4, d=128, H=8, P=16, pages=10, kv=FAKE, err=None):
+    return tq.tq_cache(fmt, d, H, P, pages, kv, err)
 
 
 def qa(c, k=FAKE, v=FAKE, s=FAKE, n=4, bits=None):
@@ -76,8 +76,8 @@ def test_quantize_append_validation():
     assert qa(desc(P=24)) == U
     assert qa(desc(H=0)) == I
     assert qa(desc(pages=0)) == I
-    assert qa(desc(kp=None)) == I
-    assert qa(desc(kp=FAKE + 8)) == I                 # 16-byte alignment
+    assert qa(desc(kv=None)) == I
+    assert qa(desc(kv=FAKE + 8)) == I                 # 16-byte alignment
     assert qa(desc(), k=None) == I
     assert qa(desc(), v=FAKE + 2) == I
     assert qa(desc(), s=FAKE + 4) == I
