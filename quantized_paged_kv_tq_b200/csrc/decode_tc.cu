@@ -140,15 +140,17 @@ __device__ __forceinline__ void pairs3(uint32_t g, uint32_t* o)
     o[3] = mk(and_or(sel3, 0x01C001C0u, kMagicTc), mul[2], add[2]);
 }
 
-// K row of one token (128 codes) -> tensor memory columns [col, col + 64).
+// K row of one token (128 codes; 16-byte chunks permuted by `sw`, see
+// k_swizzle) -> tensor memory columns [col, col + 64).
 template <int BITS>
-__device__ __forceinline__ void k_row_to_tmem(const uint8_t* row, uint32_t taddr)
+__device__ __forceinline__ void k_row_to_tmem(const uint8_t* row, uint32_t taddr, int sw)
 {
     uint32_t o[16];
+    auto chunk = [&](int c) { return *reinterpret_cast<const uint4*>(row + 16 * (c ^ sw)); };
     if constexpr (BITS == 4) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const uint4 w = *reinterpret_cast<const uint4*>(row + 16 * q);
+            const uint4 w = chunk(q);
             pairs4(w.x, o);
             pairs4(w.y, o + 4);
             pairs4(w.z, o + 8);
@@ -158,8 +160,8 @@ __device__ __forceinline__ void k_row_to_tmem(const uint8_t* row, uint32_t taddr
     } else if constexpr (BITS == 8) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const uint4 a = *reinterpret_cast<const uint4*>(row + 32 * q);
-            const uint4 b = *reinterpret_cast<const uint4*>(row + 32 * q + 16);
+            const uint4 a = chunk(2 * q);
+            const uint4 b = chunk(2 * q + 1);
             pairs8(a.x, o); pairs8(a.y, o + 2); pairs8(a.z, o + 4); pairs8(a.w, o + 6);
             pairs8(b.x, o + 8); pairs8(b.y, o + 10); pairs8(b.z, o + 12); pairs8(b.w, o + 14);
             tmem_st16(taddr + 16 * q, o);
@@ -167,7 +169,7 @@ __device__ __forceinline__ void k_row_to_tmem(const uint8_t* row, uint32_t taddr
     } else if constexpr (BITS == 2) {
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-            const uint4 w = *reinterpret_cast<const uint4*>(row + 16 * q);
+            const uint4 w = chunk(q);
             pairs2(w.x, o);
             pairs2(w.y, o + 8);
             tmem_st16(taddr + 32 * q, o);
@@ -567,7 +569,7 @@ k_decode_tc(const TcArgs a)
         const int pg = tid >> a.lp, row = tid & (P - 1);
         const uint8_t* kblk = st + pg * 2 * a.block_bytes;     // stage: [page][K block, V block]
         const uint8_t* vblk = kblk + a.block_bytes;
-        k_row_to_tmem<BITS>(kblk + row * F::CB, t_lane);
+        k_row_to_tmem<BITS>(kblk + row * F::CB, t_lane, k_swizzle<BITS>(row));
         float ks = reinterpret_cast<const float*>(kblk + P * F::CB)[row] * kinv;
         float vs = reinterpret_cast<const float*>(vblk + P * F::CB)[row] * kinv;
         const int tok = tok0 + tid;
@@ -1427,12 +1429,14 @@ cudaError_t launch_i8(const TcArgs& a, dim3 grid, cudaStream_t stream)
 
 }  // namespace
 
-// Query rows of one tensor-core CTA.  The integer kernel (2-, 4- and 8-bit
-// codes) takes 4 or 8; the f16 kernel (3-bit codes) 4, 8 or 16.
+// Query rows of one tensor-core CTA: 4, 8 or 16.  Up to 8 rows, 2-, 4- and
+// 8-bit codes go to the integer kernel; 3-bit codes, and every format with
+// more than 8 rows per kv head, to the f16 kernel (16 rows in one CTA, so
+// the kv head's pages are read once).
 int decode_tc_rows(int format, int G)
 {
-    if (format == 3) return G <= 4 ? 4 : (G <= 8 ? 8 : 16);
-    return G <= 4 ? 4 : 8;
+    (void)format;
+    return G <= 4 ? 4 : (G <= 8 ? 8 : 16);
 }
 
 cudaError_t launch_decode_tc(const void* q, const tq_cache& c, int64_t block_bytes,
@@ -1472,7 +1476,10 @@ cudaError_t launch_decode_tc(const void* q, const tq_cache& c, int64_t block_byt
         a.ws_o = reinterpret_cast<float*>(w + cnt + ml);
     }
     const dim3 grid((unsigned)a.max_splits, (unsigned)(c.num_kv_heads * a.R), (unsigned)batch);
-#define TQ_I8(B) return rows == 4 ? launch_i8<B, 4>(a, grid, stream) : launch_i8<B, 8>(a, grid, stream)
+#define TQ_I8(B)                                                                    \
+    return rows == 4   ? launch_i8<B, 4>(a, grid, stream)                              \
+           : rows == 8 ? launch_i8<B, 8>(a, grid, stream)                              \
+                       : launch_tc<B, 16>(a, grid, stream)
     switch (c.format) {
     case 2: TQ_I8(2);
     case 3:

@@ -117,18 +117,16 @@ def _expected_workspace(batch, Hkv, G, seq, P, fmt):
     """Workspace layout the decode kernels use: merge counters, then (m, l)
     and the 128-float partial output of every (unit, split, row), where a
     unit is one (sequence, kv head, row group).  Rows per CTA: 8 for the bf16
-    cache; 4 or 8 for turbo2/4/8; 4, 8 or 16 for turbo3.  Splits are 2048
-    tokens (1024 with 64-token pages)."""
+    cache; 4, 8 or 16 for the turbo formats.  Splits are 2048 tokens (1024
+    with 64-token pages)."""
     split = 1024 if P == 64 else 2048
     nsplit = -(-seq // split)
     if nsplit <= 1:
         return 0
     if fmt == 16:
         rows = 8
-    elif fmt == 3:
-        rows = 4 if G <= 4 else (8 if G <= 8 else 16)
     else:
-        rows = 4 if G <= 4 else 8
+        rows = 4 if G <= 4 else (8 if G <= 8 else 16)
     units = batch * Hkv * -(-G // rows)
     r256 = lambda x: -(-x // 256) * 256
     return r256(units * 4) + r256(units * nsplit * rows * 8) + units * nsplit * rows * 128 * 4
