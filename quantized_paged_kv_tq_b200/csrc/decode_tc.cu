@@ -286,19 +286,21 @@ __device__ __forceinline__ void issue_tile_tc(uint8_t* stage, uint64_t* bar, con
     }
 }
 
-// The same copies spread over the CTA's 4 warps: warp w takes pages
-// w, w + 4, ...; each warp's lane 0 arrives with its own byte count (the
-// stage barrier counts 4 arrivals), so no warp waits on another to issue.
+// The same copies spread over warps 1..3 (warp 0 issues S = K q'' at that
+// point): warp w takes pages w - 1, w + 2, w + 5, ...; each warp's lane 0
+// arrives with its own byte count (the stage barrier counts 4 arrivals, warp
+// 0 with none), so no warp waits on another to issue.
 __device__ __forceinline__ void issue_tile_warps(uint8_t* stage, uint64_t* bar, const TcArgs& a,
                                                  const int* pids, int kvh, int ntok, int warp,
                                                  int lane)
 {
     const int npg = (ntok + (1 << a.lp) - 1) >> a.lp;
-    const int mine = npg > warp ? (npg - warp + 3) >> 2 : 0;      // pages of this warp
+    const int first = warp - 1;
+    const int mine = (warp > 0 && npg > first) ? (npg - first + 2) / 3 : 0;   // pages of this warp
     if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(2 * mine * a.block_bytes));
     __syncwarp();
     if (lane < mine) {
-        const int j = warp + 4 * lane;
+        const int j = first + 3 * lane;
         int pid = pids[j];
         if (pid < 0 || pid >= a.num_pages) {
             report_error(a.err, TQ_ERR_DEVICE_CHECK, kErrPageRange);
@@ -1186,7 +1188,7 @@ k_decode_i8(const TcArgs a)
     };
     // One thread issues the 4 K-steps of a product and commits them: MMAs
     // accumulating into one tensor-memory accumulator stay in one thread's
-    // issue order.
+    // issue order (S from thread 0, O from thread 96).
     auto issue_qk = [&]() {
         tc_fence_after();
 #pragma unroll
@@ -1352,8 +1354,8 @@ k_decode_i8(const TcArgs a)
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
-        // h. O^T += V^T P''
-        if (tid == 0) issue_pv();
+        // h. O^T += V^T P'' (warp 3, which issued the fewest copies)
+        if (tid == 96) issue_pv();
         o_acc = true;
     }
 
