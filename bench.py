@@ -224,10 +224,11 @@ def run_reference(args):
     fmt = args.fmt or w.formats[0]
     budget = 90.0
     # calibrate the per-step sample so the whole run stays within ~budget
-    dt, b = oracle_sample_decode(w, fmt, 1024)
-    per_tok = dt / 1024
+    ncal = min(1024, int(w.seq_lens[0]))
+    dt, b = oracle_sample_decode(w, fmt, ncal)
+    per_tok = dt / ncal
     ntok = int(max(16, min(int(w.seq_lens[0]), budget / (args.steps + args.warmup) / per_tok)))
-    ntok = (ntok // 16) * 16
+    ntok = max(16, (ntok // 16) * 16)
     for i in range(args.warmup):
         oracle_sample_decode(w, fmt, ntok, i % w.num_kv_heads)
     secs, nbytes = 0.0, 0
