@@ -44,10 +44,9 @@
  * Ownership.  The library allocates nothing and keeps no state between calls
  * (the one exception is the fixed scratch array of tq_paged_decode_noalloc,
  * described there).  Every buffer is caller-owned device memory unless
- * stated otherwise.  Every
- * call is asynchronous on the given CUDA stream (a cudaStream_t passed as
- * void*, NULL = legacy default stream); calls on different streams are safe
- * when their buffers are disjoint.
+ * stated otherwise.  Every call is asynchronous on the given CUDA stream (a
+ * cudaStream_t passed as void*, NULL = legacy default stream); calls on
+ * different streams are safe when their buffers are disjoint.
  *
  * Errors.  Arguments are checked on the host before anything is launched; a
  * failed check returns a status and launches nothing.  A CUDA launch failure
