@@ -90,12 +90,22 @@ def measured_peaks():
 DECODE_SOURCES = ("decode.cu", "decode_tc.cu", "tq_device.cuh")
 
 
+def _code_only(src: str) -> str:
+    """C/CUDA source without comments, blank lines or trailing blanks, so a
+    comment edit does not change the fingerprint of the code."""
+    import re
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+
+
 def decode_sources_sha256() -> str:
-    """sha256 over the decode kernels' sources, in DECODE_SOURCES order."""
+    """sha256 over the code (comments stripped) of the decode kernels'
+    sources, in DECODE_SOURCES order."""
     h = hashlib.sha256()
     for name in DECODE_SOURCES:
-        with open(os.path.join(ROOT, "quantized_paged_kv_tq_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "quantized_paged_kv_tq_b200", "csrc", name)) as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()
 
 
