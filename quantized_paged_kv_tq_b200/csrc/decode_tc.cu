@@ -6,11 +6,20 @@
 // every attention step.  "infero", section "Continuous batching": a running
 // batch shares the GPU over a paged KV cache.
 //
+// Two kernels share the structure below:
+//   k_decode_i8  (2-, 4- and 8-bit codes, up to 8 query rows per kv head):
+//                integer MMAs (kind::i8) on the codes as bytes; see the
+//                section "Integer tensor-core variant" further down.
+//   k_decode_tc  (3-bit codes, and any format with 9-16 rows per kv head):
+//                f16 MMAs (kind::f16) on codes unpacked to exact f16
+//                integers; described here.
+//
 // One CTA (128 threads) owns one (sequence, kv head, row group, split) with
 // splits of 2048 tokens (1024 for 64-token pages) fixed by the sequence
-// length alone.  The split is walked in tiles of 128 tokens; the K and V page
-// blocks of a tile arrive by 1-D bulk async copies into a 2-stage ring.
-// Per tile:
+// length alone.  The split is walked in tiles of 128 tokens; each page of a
+// tile (its adjacent K and V blocks) arrives by one 1-D bulk async copy into
+// a 2-stage ring.
+// Per tile (k_decode_tc):
 //   1. thread t unpacks token t's K codes into exact f16 integers and stores
 //      them into tensor memory (lane t): the A operand of S = K q'.
 //   2. one thread issues S[128 tok][N] = A x Q' (Q' in shared memory: the
