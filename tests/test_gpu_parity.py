@@ -93,10 +93,12 @@ def test_quantize_full_size_sampled(name, fmt):
 # ---------------------------------------------------------------- decode
 @pytest.mark.parametrize("fmt", TURBO + (16,))
 @pytest.mark.parametrize("q_len,Hq,Hkv", [(1, 8, 2), (1, 10, 2), (4, 8, 2), (3, 6, 1),
-                                          (1, 16, 1), (8, 64, 8)])
+                                          (1, 16, 1), (8, 64, 8), (2, 4, 2), (2, 8, 2)])
 def test_decode_small(fmt, q_len, Hq, Hkv):
     """Ragged lengths (2600 = 2 splits + tail, 37 < one tile, 2049 = one
-    token past a split), 1-8 query rows per kv head up to 16 and 64."""
+    token past a split), 1-8 query rows per kv head up to 16 and 64; q_len 2
+    with 4 and 8 rows per kv head takes the causal path of the 4- and 8-row
+    kernels, q_len 3-8 with more rows that of the 16-row one."""
     w = small(fmt, q_len=q_len, num_q_heads=Hq, num_kv_heads=Hkv,
               seq_lens=(2600, 37 + q_len, 2049))
     cache = gpu_fill(w, fmt)
@@ -201,10 +203,12 @@ def test_append_order_independence():
         assert torch.equal(a.k_pages, x.k_pages) and torch.equal(a.v_pages, x.v_pages)
 
 
-def test_causal_last_split_fully_masked_rows():
-    """seq_len 2050 with q_len 4: the second split holds keys 2048-2049
-    only, which rows t = 0, 1 must not see (their partial is empty)."""
-    w = small(4, q_len=4, seq_lens=(2050, 2052))
+@pytest.mark.parametrize("q_len,lens", [(4, (2050, 2052)), (2, (2049, 2050))])
+def test_causal_last_split_fully_masked_rows(q_len, lens):
+    """q_len 4 at seq_len 2050 (16 rows per kv head): the second split holds
+    keys 2048-2049 only, which rows t = 0, 1 must not see (their partial is
+    empty); q_len 2 at 2049 (8 rows): row t = 0 sees nothing of key 2048."""
+    w = small(4, q_len=q_len, seq_lens=lens)
     cache = gpu_fill(w, 4)
     check_close(gpu_decode(w, 4, cache), oracle_decode(w, 4, np.arange(2)))
 
