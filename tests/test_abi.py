@@ -162,3 +162,42 @@ def test_read_device_error_without_word():
     assert tq.lib().tq_read_device_error(ctypes.byref(desc(err=None)), ctypes.byref(code), 1,
                                          None) == 0
     assert code.value == 0
+
+
+def test_descriptor_layout_matches_the_c_header(tmp_path):
+    """The ctypes descriptor has the size and field offsets a C compiler
+    gives tq_cache, and the enum values the header defines."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "layout.c"
+    src.write_text(
+        '#include <stddef.h>\n#include <stdio.h>\n#include "tq.h"\n'
+        "int main(void) {\n"
+        '  printf("%zu %zu %zu %zu %zu %zu %zu %zu\\n", sizeof(tq_cache),\n'
+        "         offsetof(tq_cache, format), offsetof(tq_cache, head_dim),\n"
+        "         offsetof(tq_cache, num_kv_heads), offsetof(tq_cache, page_size),\n"
+        "         offsetof(tq_cache, num_pages), offsetof(tq_cache, pages),\n"
+        "         offsetof(tq_cache, dev_error));\n"
+        '  printf("%d %d %d %d %d %d\\n", TQ_TURBO2, TQ_TURBO3, TQ_TURBO4, TQ_TURBO8, TQ_BF16,\n'
+        "         TQ_ABI_VERSION);\n"
+        '  printf("%d %d %d %d %d %d %d\\n", TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED,\n'
+        "         TQ_ERR_CUDA, TQ_ERR_TIMEOUT, TQ_ERR_DEVICE_CHECK, TQ_ERR_WORKSPACE);\n"
+        "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.check_call([cc, "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o",
+                           str(exe)])
+    lines = subprocess.check_output([str(exe)], text=True).split("\n")
+    sizes = [int(x) for x in lines[0].split()]
+    C = tq.tq_cache
+    assert sizes[0] == ctypes.sizeof(C)
+    assert sizes[1:] == [getattr(C, f).offset for f in
+                         ("format", "head_dim", "num_kv_heads", "page_size", "num_pages",
+                          "pages", "dev_error")]
+    assert [int(x) for x in lines[1].split()] == [tq.TQ_TURBO2, tq.TQ_TURBO3, tq.TQ_TURBO4,
+                                                  tq.TQ_TURBO8, tq.TQ_BF16, tq.abi_version()]
+    assert [int(x) for x in lines[2].split()] == [
+        tq.TQ_OK, tq.TQ_ERR_INVALID_ARG, tq.TQ_ERR_UNSUPPORTED, tq.TQ_ERR_CUDA,
+        tq.TQ_ERR_TIMEOUT, tq.TQ_ERR_DEVICE_CHECK, tq.TQ_ERR_WORKSPACE]
