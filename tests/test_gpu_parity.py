@@ -115,6 +115,17 @@ def test_decode_page64(fmt):
     check_close(gpu_decode(w, fmt, cache), oracle_decode(w, fmt, np.arange(w.batch)))
 
 
+@pytest.mark.parametrize("fmt", TURBO + (16,))
+@pytest.mark.parametrize("q_len", [1, 4])
+def test_decode_page32(fmt, q_len):
+    """32-token pages: 4 pages per 128-token tile, 4 and 16 rows per kv head."""
+    w = small(fmt, page_size=32, q_len=q_len, seq_lens=(2600, 40 + q_len, 2049))
+    cache = gpu_fill(w, fmt)
+    check_close(gpu_decode(w, fmt, cache), oracle_decode(w, fmt, np.arange(w.batch)),
+                f"fmt {fmt} page 32 q_len {q_len}")
+    assert cache.read_error() == 0
+
+
 CONFIG_RUNS = [("tiny", 4, None), ("batch8", 4, (0, 5)), ("cbatch64", 3, "minmax"),
                ("cbatch64", 8, "minmax"), ("cbatch64", 16, "minmax"),
                ("target64x8k", 4, (0, 63)), ("long128k", 4, (2,)), ("long128k", 2, (1,)),
