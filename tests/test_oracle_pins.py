@@ -175,6 +175,93 @@ def test_round_half_away_from_zero_at_ties():
     assert list(c[:3]) == [127, 3, -127]
 
 
+def _fl32(q):
+    """Nearest fp32 (ties to even) of an exact rational q (normal range)."""
+    from fractions import Fraction
+    if q == 0:
+        return Fraction(0)
+    sgn = -1 if q < 0 else 1
+    a = abs(q)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    ulp = Fraction(2) ** (e - 23)
+    m = a / ulp
+    n = m.numerator // m.denominator
+    rem = m - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    return sgn * n * ulp
+
+
+def _round_half_away(q):
+    from fractions import Fraction
+    sgn = -1 if q < 0 else 1
+    a = abs(q)
+    n = a.numerator // a.denominator
+    return sgn * (n + (1 if a - n >= Fraction(1, 2) else 0))
+
+
+def test_division_order_golden():
+    """fl32(y L) / s with an IEEE division, not y fl32(L / s) nor
+    fl32(y / s) L: on each fixture row the three orders give different
+    codes; the expected one is derived again here with exact rationals."""
+    from fractions import Fraction
+    rows = read_golden("quant_division_order.txt")
+    assert len(rows) >= 9
+    for bits_s, y_hex, s_hex, code_s, other_s in rows:
+        bits, L = int(bits_s), Lof(int(bits_s))
+        y = np.uint32(int(y_hex, 16)).view(np.float32)
+        s = np.uint32(int(s_hex, 16)).view(np.float32)
+        Y, S = Fraction(float(y)), Fraction(float(s))
+        want = _round_half_away(_fl32(_fl32(Y * L) / S))
+        recip = _round_half_away(_fl32(Y * _fl32(Fraction(L) / S)))
+        late = _round_half_away(_fl32(_fl32(Y / S) * L))
+        assert want == int(code_s) and recip == late == int(other_s) != want
+        vec = np.zeros(128, np.float32)
+        vec[0], vec[1], vec[2] = s, y, -y
+        codes, scale = oracle.quantize_rotated(vec, bits)
+        assert scale == s and codes[0] == L
+        assert codes[1] == want and codes[2] == -want
+
+
+@pytest.mark.parametrize("bits,y,s,code", [(4, 1.25, 3.5, 3), (3, 1.25, 1.5, 3),
+                                           (8, 0.25, 5.0, 6), (2, 0.75, 1.5, 1)])
+def test_exact_ties_with_scale_not_L(bits, y, s, code):
+    """Ties y L / s = n + 1/2 that are exact at every fp32 step with s != L
+    (and s not a power of two for turbo4/3/8): 1.25*7/3.5 = 2.5 -> 3,
+    1.25*3/1.5 = 2.5 -> 3, 0.25*127/5 = 6.35 -> 6 (no tie, a plain case),
+    0.75*1/1.5 = 0.5 -> 1; negatives mirror them."""
+    vec = np.zeros(128, np.float32)
+    vec[0], vec[1], vec[2] = s, y, -y
+    codes, scale = oracle.quantize_rotated(vec, bits)
+    assert scale == np.float32(s) and list(codes[1:3]) == [code, -code]
+
+
+def test_fwht_stage_order_golden():
+    """Strides 1, 2, 4 in that order, each butterfly rounded to fp32: the
+    hand-derived d = 8 fixture differs bit for bit from the reverse order
+    (and from the exact transform)."""
+    want = np.array([int(h, 16) for _, h in read_golden("fwht_stage_order_d8.txt")],
+                    np.uint32).view(np.float32)
+    x = np.array([1.0, 2.0 ** -24, -1.0, 2.0 ** -24, 0, 0, 0, 0], np.float32)
+    got = oracle.fwht_f32(x)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+    # the rotation: the same butterflies, then one multiply by fp32(1/sqrt(8))
+    c = np.float32(1 / math.sqrt(8))
+    y = oracle.rotate_f32(W.f32_to_bf16_bits(x))
+    assert np.array_equal(y.view(np.uint32), (want * c).view(np.uint32))
+    # embedded in a 128-vector: strides 8..64 only meet zeros, so entries
+    # 0..7 carry the same values and entries 8i..8i+7 copy them
+    x128 = np.zeros(128, np.float32)
+    x128[:8] = x
+    y128 = oracle.rotate_f32(W.f32_to_bf16_bits(x128))
+    c128 = np.float32(1 / math.sqrt(128))
+    assert np.array_equal(y128.view(np.uint32), np.tile(want * c128, 16).view(np.uint32))
+
+
 @pytest.mark.parametrize("bits", BITS)
 def test_packing_matches_numpy_little_endian_bits(bits):
     rng = np.random.default_rng(30 + bits)
