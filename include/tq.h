@@ -54,7 +54,8 @@
  * slot outside the pool, a sequence length outside [q_len, max_seq_len], a
  * bounded wait that expired) skip the affected work and record the first
  * such event in the optional device word cache->dev_error; read it with
- * tq_read_device_error.  No device code traps or asserts.
+ * tq_read_device_error.  The outputs of a call that recorded an event are
+ * unspecified for the affected sequences.  No device code traps or asserts.
  *
  * Supported shapes: head_dim 128; page_size 16, 32 or 64; 1 <= q_len and
  * q_len * (num_q_heads / num_kv_heads) <= 64.
@@ -158,7 +159,9 @@ size_t tq_decode_workspace_size(int32_t batch, int32_t q_len,
 
 /*
  * tq_decode_workspace_init -- zero the merge counters of a workspace.  Call
- * once after allocating it; every decode call leaves them zero again.
+ * once after allocating it; every decode call leaves them zero again, a call
+ * whose device word reports TQ_ERR_TIMEOUT included (a split that gives up
+ * records an empty partial and still takes its turn in the merge).
  */
 tq_status tq_decode_workspace_init(void* workspace, size_t workspace_bytes,
                                    void* stream);

@@ -86,10 +86,16 @@ tq_status check_append(const void* k, const void* v, const int64_t* slots, int32
     return TQ_OK;
 }
 
-tq_status check_decode(const void* q, const tq_cache* c, const int32_t* page_table,
-                       int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
-                       int32_t q_len, int32_t num_q_heads, int32_t max_seq_len, const float* out,
-                       const void* workspace, size_t workspace_bytes, bool turbo)
+}  // namespace
+
+namespace tq {
+
+// Host checks of a decode call except its workspace, shared by every decode
+// entry point (tq_paged_decode, tq_paged_decode_bf16 and the no-alloc decode).
+tq_status check_decode_call(const void* q, const tq_cache* c, const int32_t* page_table,
+                            int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
+                            int32_t q_len, int32_t num_q_heads, int32_t max_seq_len,
+                            const float* out, bool turbo)
 {
     tq_status s = check_cache(c, turbo);
     if (s != TQ_OK) return s;
@@ -108,6 +114,28 @@ tq_status check_decode(const void* q, const tq_cache* c, const int32_t* page_tab
     if (!aligned16(q) || !aligned16(out) || (reinterpret_cast<uintptr_t>(page_table) & 3u) ||
         (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
         return TQ_ERR_INVALID_ARG;
+    return TQ_OK;
+}
+
+// Bytes of one K (or V) block; 0 for an unsupported combination.
+int64_t cache_block_bytes(int32_t format, int32_t head_dim, int32_t page_size)
+{
+    return block_bytes(format, head_dim, page_size);
+}
+
+}  // namespace tq
+
+namespace {
+
+tq_status check_decode(const void* q, const tq_cache* c, const int32_t* page_table,
+                       int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
+                       int32_t q_len, int32_t num_q_heads, int32_t max_seq_len, const float* out,
+                       const void* workspace, size_t workspace_bytes, bool turbo)
+{
+    tq_status s = tq::check_decode_call(q, c, page_table, max_pages_per_seq, seq_lens, batch,
+                                        q_len, num_q_heads, max_seq_len, out, turbo);
+    if (s != TQ_OK || batch == 0) return s;
+    const int64_t G = (int64_t)q_len * (num_q_heads / c->num_kv_heads);
     const size_t need = tq::decode_workspace_bytes(batch, c->num_kv_heads, (int)G, max_seq_len,
                                                    c->page_size, c->format);
     if (need > 0) {

@@ -521,7 +521,11 @@ k_decode(const DecodeArgs a)
             }
     }
     __syncthreads();
-    if (sFlag[0]) return;
+    // A CTA that gave up on a bounded wait (sFlag[0], CTA-uniform here) reads
+    // none of its partials; in a multi-split sequence it still records an
+    // empty partial and takes its ticket, so the counter wraps back to zero.
+    const bool valid = sFlag[0] == 0;
+    if (!valid && nsplit == 1) return;
 
     // ---- merge the 4 warps; warp w takes rows w and w + 4
     const int nrows = min(kRowsPerCta, min(4 * NT, a.G - rg * kRowsPerCta));
@@ -531,6 +535,10 @@ k_decode(const DecodeArgs a)
     for (int k = 0; k < 2; ++k) {
         const int rr = warp + 4 * k;
         if (rr >= nrows) continue;
+        if (!valid) {
+            if (lane == 0) a.ws_ml[part * kRowsPerCta + rr] = make_float2(-CUDART_INF_F, 0.f);
+            continue;
+        }
         float M = -CUDART_INF_F;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sM[w * kRowsPerCta + rr]);
@@ -586,7 +594,8 @@ k_decode(const DecodeArgs a)
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         for (int sp = 0; sp < nsplit; ++sp) {
             const float2 ml = __ldcg(a.ws_ml + (base + sp) * kRowsPerCta + rr);
-            const float sc = ml.x == -CUDART_INF_F ? 0.f : exp2f(ml.x - M);
+            if (ml.x == -CUDART_INF_F) continue;       // empty split: no keys, no O written
+            const float sc = exp2f(ml.x - M);
             Lsum += sc * ml.y;
             const float4 v = __ldcg(reinterpret_cast<const float4*>(
                 a.ws_o + ((base + sp) * kRowsPerCta + rr) * kHeadDim) + lane);

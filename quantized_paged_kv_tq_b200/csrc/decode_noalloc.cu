@@ -24,6 +24,11 @@
 #define TQ_API extern "C" __attribute__((visibility("default")))
 
 namespace tq {
+tq_status check_decode_call(const void* q, const tq_cache* c, const int32_t* page_table,
+                            int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
+                            int32_t q_len, int32_t num_q_heads, int32_t max_seq_len,
+                            const float* out, bool turbo);
+int64_t cache_block_bytes(int32_t format, int32_t head_dim, int32_t page_size);
 size_t decode_workspace_bytes(int batch, int num_kv_heads, int G, int max_seq_len,
                               int page_size, int format);
 int decode_row_groups(int format, int G);
@@ -66,8 +71,6 @@ cudaError_t scratch_on_current_device(void** out)
     return cudaSuccess;
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
 
 TQ_API tq_status tq_paged_decode_noalloc(const void* q, const tq_cache* cache,
@@ -76,33 +79,13 @@ TQ_API tq_status tq_paged_decode_noalloc(const void* q, const tq_cache* cache,
                                          int32_t num_q_heads, int32_t max_seq_len, float* out,
                                          void* stream)
 {
-    // the same host checks as tq_paged_decode, then the scratch-size limit
-    if (!cache) return TQ_ERR_INVALID_ARG;
+    // the same host checks as tq_paged_decode (one shared function), then
+    // the scratch-size limit in place of the workspace checks
+    const tq_status st = tq::check_decode_call(q, cache, page_table, max_pages_per_seq, seq_lens,
+                                               batch, q_len, num_q_heads, max_seq_len, out, true);
+    if (st != TQ_OK || batch == 0) return st;
     const int f = cache->format;
-    if (f != TQ_TURBO2 && f != TQ_TURBO3 && f != TQ_TURBO4 && f != TQ_TURBO8)
-        return TQ_ERR_INVALID_ARG;
-    if (cache->head_dim <= 0 || cache->page_size <= 0 || cache->num_kv_heads <= 0 ||
-        cache->num_pages <= 0)
-        return TQ_ERR_INVALID_ARG;
-    if (cache->head_dim != 128) return TQ_ERR_UNSUPPORTED;
-    if (cache->page_size != 16 && cache->page_size != 32 && cache->page_size != 64)
-        return TQ_ERR_UNSUPPORTED;
-    if (!cache->pages || !aligned16(cache->pages) ||
-        (reinterpret_cast<uintptr_t>(cache->dev_error) & 3u))
-        return TQ_ERR_INVALID_ARG;
-    if (batch < 0 || q_len <= 0 || num_q_heads <= 0 || max_seq_len <= 0) return TQ_ERR_INVALID_ARG;
-    if (num_q_heads % cache->num_kv_heads || max_seq_len < q_len) return TQ_ERR_INVALID_ARG;
-    if (max_pages_per_seq < ((int64_t)max_seq_len + cache->page_size - 1) / cache->page_size)
-        return TQ_ERR_INVALID_ARG;
     const int64_t G = (int64_t)q_len * (num_q_heads / cache->num_kv_heads);
-    if (G > 64 || batch > 65535) return TQ_ERR_UNSUPPORTED;
-    if ((int64_t)cache->num_kv_heads * tq::decode_row_groups(f, (int)G) > 65535)
-        return TQ_ERR_UNSUPPORTED;
-    if (batch == 0) return TQ_OK;
-    if (!q || !page_table || !seq_lens || !out || !aligned16(q) || !aligned16(out) ||
-        (reinterpret_cast<uintptr_t>(page_table) & 3u) ||
-        (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
-        return TQ_ERR_INVALID_ARG;
 
     const size_t need = tq::decode_workspace_bytes(batch, cache->num_kv_heads, (int)G,
                                                    max_seq_len, cache->page_size, f);
@@ -120,8 +103,7 @@ TQ_API tq_status tq_paged_decode_noalloc(const void* q, const tq_cache* cache,
         if (cudaMemsetAsync(scratch, 0, units * sizeof(uint32_t), s) != cudaSuccess)
             return TQ_ERR_CUDA;
     }
-    const int64_t bits = f;
-    const int64_t block = (int64_t)cache->page_size * (128 * bits / 8 + 4);
+    const int64_t block = tq::cache_block_bytes(f, cache->head_dim, cache->page_size);
     const cudaError_t e = tq::launch_decode(q, *cache, block, page_table, max_pages_per_seq,
                                             seq_lens, batch, q_len, num_q_heads, max_seq_len,
                                             out, scratch, s);

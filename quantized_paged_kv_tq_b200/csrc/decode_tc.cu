@@ -334,16 +334,25 @@ __device__ __forceinline__ void load_split_pids(int* s_pid, const TcArgs& a, int
 // row sums [4][16]; m_run: row maxima (log2 units).  A split that is the whole
 // sequence normalises, rotates back and writes; otherwise the partial goes to
 // the workspace and the last split CTA of the unit (atomic ticket) merges.
+// valid == false (the CTA gave up on a bounded wait; CTA-uniform): nothing
+// is read from sO, s_l or m_run; a split of a longer sequence still records
+// an empty partial (m = -inf) and takes its ticket, so the unit's counter
+// wraps back to zero and the workspace stays usable for later calls.
 template <int RG>
 __device__ __forceinline__ void tc_finish(const TcArgs& a, const float* sO, const float* s_l,
                                           const float* m_run, int* s_flag, int b, int kvh, int rg,
                                           int split, int nsplit, int nrows, int warp, int lane,
-                                          int tid)
+                                          int tid, bool valid)
 {
     const int64_t unit = ((int64_t)b * gridDim.y + blockIdx.y);
     const int64_t part = unit * a.max_splits + split;
     const float rs = 0.08838834764831845f;
+    if (!valid && nsplit == 1) return;
     for (int rr = warp; rr < nrows; rr += 4) {
+        if (!valid) {
+            if (lane == 0) a.ws_ml[part * RG + rr] = make_float2(-CUDART_INF_F, 0.f);
+            continue;
+        }
         const float M = m_run[rr];
         const float Lsum = s_l[rr] + s_l[16 + rr] + s_l[32 + rr] + s_l[48 + rr];
         float x[4];
@@ -386,7 +395,8 @@ __device__ __forceinline__ void tc_finish(const TcArgs& a, const float* sO, cons
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         for (int sp = 0; sp < nsplit; ++sp) {
             const float2 ml = __ldcg(a.ws_ml + (base + sp) * RG + rr);
-            const float sc = ml.x == -CUDART_INF_F ? 0.f : exp2f(ml.x - M);
+            if (ml.x == -CUDART_INF_F) continue;       // empty split: no keys, no O written
+            const float sc = exp2f(ml.x - M);
             Lsum += sc * ml.y;
             const float4 v = __ldcg(reinterpret_cast<const float4*>(
                 a.ws_o + ((base + sp) * RG + rr) * kHeadDim) + lane);
@@ -716,9 +726,12 @@ k_decode_tc(const TcArgs a)
         }
     }
 
-    // ---- epilogue: O rows into shared memory, l summed over the CTA
+    // ---- epilogue: O rows into shared memory, l summed over the CTA.  The
+    // decision to finish is taken for the whole CTA (warp-collective tensor
+    // memory loads and the barriers of tc_finish follow).
     bool ok = !aborted && mbar_wait_sleep(bar_o, (uint32_t)((ntiles - 1) & 1), kPollsTc);
     tc_fence_after();
+    ok = __syncthreads_and(ok);
     const int nrows = min(RG, a.G - rg * RG);
     float* sO = reinterpret_cast<float*>(ring);          // [RG][128]
     if (ok) {
@@ -746,9 +759,8 @@ k_decode_tc(const TcArgs a)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
-    if (!ok) return;
-
-    tc_finish<RG>(a, sO, s_l, m_run, s_flag, b, kvh, rg, split, nsplit, nrows, warp, lane, tid);
+    tc_finish<RG>(a, sO, s_l, m_run, s_flag, b, kvh, rg, split, nsplit, nrows, warp, lane, tid,
+                  ok);
 }
 
 // ===================================================================
@@ -1396,8 +1408,8 @@ k_decode_i8(const TcArgs a)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
-    if (!ok) return;
-    tc_finish<RG>(a, sO, s_l, m_run, s_flag, b, kvh, rg, split, nsplit, nrows, warp, lane, tid);
+    tc_finish<RG>(a, sO, s_l, m_run, s_flag, b, kvh, rg, split, nsplit, nrows, warp, lane, tid,
+                  ok);
 }
 
 template <int BITS, int RG>

@@ -6,7 +6,10 @@ reserves all of its device memory at start-up.  For them the library keeps
 the split-KV scratch in a fixed array of its own.  This test calls that
 entry point through the C ABI and checks its output against the regular
 tq_paged_decode (caller-provided workspace) on two calls in a row, the
-second one reusing the scratch the first one left behind.
+second one reusing the scratch the first one left behind.  Both entry
+points launch the same kernel with the same fixed splits and the same merge
+order, so the outputs must agree bit for bit; the no-alloc output is also
+checked against the CPU oracle's fp64 result at the parity tolerances.
 
 The file name sorts last so that, in a run that stops at the first failure,
 every other test has already run; it also builds and sets up everything it
@@ -24,12 +27,24 @@ ATOL = 2e-3      # the tolerances the parity tests use
 RTOL_L2 = 1e-3
 
 
-def _close(a, b):
-    a = a.double()
-    b = b.double()
-    assert torch.isfinite(a).all()
-    assert (a - b).abs().max().item() <= ATOL
-    assert ((a - b).norm() / b.norm()).item() <= RTOL_L2
+def _close(got: np.ndarray, ref: np.ndarray):
+    got = got.astype(np.float64)
+    assert np.all(np.isfinite(got))
+    assert np.abs(got - ref).max() <= ATOL
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) <= RTOL_L2
+
+
+def _oracle_decode(w, fmt):
+    """fp64 oracle output from a cache the oracle builds itself from the
+    same generator values (never from GPU output)."""
+    import oracle
+    bb = oracle.block_bytes(fmt, w.head_dim, w.page_size)
+    kp = np.zeros((w.num_pages, w.num_kv_heads, bb), np.uint8)
+    vp = np.zeros_like(kp)
+    for slots, k, v in w.iter_fill():
+        oracle.quantize_append(k, v, slots, fmt, w.page_size, kp, vp)
+    return oracle.paged_decode(w.queries(), fmt, w.page_size, kp, vp, w.page_table,
+                               w.seq_lens, w.num_kv_heads)
 
 
 def test_noalloc_matches_workspace_decode_twice():
@@ -57,6 +72,7 @@ def test_noalloc_matches_workspace_decode_twice():
         ref = torch.full(shape, float("nan"), device="cuda")
         tq.tq_paged_decode(q, cache, pt, sl, q_len, ref, max_seq_len=w.max_seq_len)
         stream = torch.cuda.current_stream().cuda_stream
+        torch.cuda.synchronize()
         for _ in range(2):
             out = torch.full(shape, float("nan"), device="cuda")
             st = tq.lib().tq_paged_decode_noalloc(
@@ -65,8 +81,9 @@ def test_noalloc_matches_workspace_decode_twice():
                 stream)
             assert st == tq.TQ_OK, tq.status_string(st)
             torch.cuda.synchronize()
-            _close(out, ref)
+            assert torch.equal(out, ref)           # same kernel, splits and merge order
         assert cache.read_error() == 0
+        _close(out.cpu().numpy(), _oracle_decode(w, fmt))
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
