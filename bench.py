@@ -9,9 +9,11 @@ decode over the whole paged cache (tq_paged_decode), on the workload named in
 starts; the cache (570 MB for the default workload) is larger than L2, so no
 flush is needed between steps.  ``value`` is the effective KV bandwidth of
 the step (algorithmic cache bytes read per step / step time); the line also
-carries seq/s, the append bandwidth, a roofline object for the decode
-kernel, an end-to-end number through the C ABI with host buffers, the
-oracle as a CPU baseline, and the SM clocks seen during the timed region.
+carries seq/s, the per-step and bulk append bandwidth, a roofline object for
+the decode kernel, an end-to-end number through the C ABI with host buffers,
+the oracle as a CPU baseline, the SM clocks seen around the timed region,
+and ``per_config``: the decode and bulk append of every other synthetic
+workload and format, timed alone with the L2 flushed before every launch.
 
 With --gpus N (launched by torch.distributed.run) every rank runs an
 independent replica on its own GPU: the workload has no exchange step, so
@@ -263,6 +265,35 @@ def run_reference(args):
 
 
 # --------------------------------------------------------------- GPU arm
+# The (workload, format) pairs timed in `per_config`: every format of every
+# synthetic workload (the bench workload itself is the line's main part).
+PER_CONFIG = (("tiny", 4), ("batch8", 4), ("cbatch64", 3), ("cbatch64", 8), ("cbatch64", 16),
+              ("long128k", 4), ("long128k", 2), ("specverify", 4))
+FORMAT_NAMES = {2: "turbo2", 3: "turbo3", 4: "turbo4", 8: "turbo8", 16: "bf16"}
+L2_FLUSH_BYTES = 256 << 20         # > the 126 MB L2
+
+
+def decode_kernel_label(fmt: int, G: int) -> str:
+    """Name of the decode kernel instantiation the library launches for a
+    format and G = q_len x GQA rows per kv head (a label for the report)."""
+    if fmt == 16:
+        return "k_decode<16>"
+    rows = 4 if G <= 4 else (8 if G <= 8 else 16)
+    if fmt == 3 or rows == 16:
+        return f"k_decode_tc<{fmt},{rows}>"
+    return f"k_decode_i8<{fmt},{rows}>"
+
+
+def append_bytes(tokens: int, num_kv_heads: int, fmt: int, head_dim: int = 128) -> int:
+    """Algorithmic bytes of appending `tokens` tokens: bf16 K and V read,
+    codes and scales (or bf16 rows) written, one int64 slot read."""
+    return tokens * (num_kv_heads * 2 * (2 * head_dim + W.row_bytes(fmt)) + 8)
+
+
+def median(xs):
+    return statistics.median(xs) if xs else float("nan")
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -282,25 +313,81 @@ def run_ours(args):
     tqbuild.build()
     from quantized_paged_kv_tq_b200 import tq
 
-    w = W.make(args.workload)
-    fmt = args.fmt or w.formats[0]
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
+    peaks, peak_kind = measured_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
 
     def d_bf16(u16):
         return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).view(
             torch.bfloat16).to(dev)
 
-    # ---- resident cache: every context token but the last of each sequence
-    cache = tq.Cache(fmt, w.num_pages, w.num_kv_heads, w.page_size, device=dev)
-    ctx = w.seq_lens - 1
-    for slots, k, v in w.iter_fill(upto=ctx):
-        ks, vs = d_bf16(k), d_bf16(v)
-        ss = torch.from_numpy(slots.astype(np.int64)).to(dev)
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    def resident_fill_inputs(w, upto=None):
+        """Every fill slot of w (positions [0, upto[b]) of each sequence) with
+        its K/V values, resident on the device: (slots, k, v)."""
+        n = len(w.fill_slots(upto))
+        k_d = torch.empty((n, w.num_kv_heads, w.head_dim), dtype=torch.bfloat16, device=dev)
+        v_d = torch.empty_like(k_d)
+        s_d = torch.empty(n, dtype=torch.int64, device=dev)
+        i = 0
+        for slots, k, v in w.iter_fill(1 << 16, upto=upto):
+            m = len(slots)
+            k_d[i:i + m] = d_bf16(k)
+            v_d[i:i + m] = d_bf16(v)
+            s_d[i:i + m] = torch.from_numpy(slots.astype(np.int64)).to(dev)
+            i += m
+        return s_d, k_d, v_d
+
+    def appender(cache, fmt):
         if fmt == 16:
-            tq.tq_append_bf16(ks, vs, ss, cache)
-        else:
-            tq.tq_quantize_append(ks, vs, ss, fmt, cache)
+            return lambda k, v, s: tq.tq_append_bf16(k, v, s, cache)
+        return lambda k, v, s: tq.tq_quantize_append(k, v, s, fmt, cache)
+
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def timed(fn, reps, flush):
+        """Median / min device time (ms) of fn over reps launches, each
+        bracketed by CUDA events on the launching stream; the L2 is flushed
+        (an untimed 256 MB write) before each one when `flush`."""
+        starts, ends = [ev() for _ in range(reps)], [ev() for _ in range(reps)]
+        for r in range(reps):
+            if flush:
+                flush_buf.zero_()
+            starts[r].record(stream)
+            fn()
+            ends[r].record(stream)
+        torch.cuda.synchronize()
+        t = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+        return median(t), min(t)
+
+    def bulk_append_report(w, fmt, fill, s_d, k_d, v_d, flush):
+        """The fill of a whole context as one append call (idempotent, so it
+        can be repeated): time and bandwidth."""
+        ms, ms_min = timed(lambda: fill(k_d, v_d, s_d), 3, flush)
+        nbytes = append_bytes(int(s_d.numel()), w.num_kv_heads, fmt)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return {"tokens": int(s_d.numel()), "us": ms * 1e3, "bytes": nbytes, "gbs": gbs,
+                "frac_of_hbm": gbs / peak}
+
+    # ================================================================ main
+    w = W.make(args.workload)
+    fmt = args.fmt or w.formats[0]
+
+    # ---- resident cache: every context token but the last of each sequence,
+    # appended by one timed bulk call
+    cache = tq.Cache(fmt, w.num_pages, w.num_kv_heads, w.page_size, device=dev)
+    fill = appender(cache, fmt)
+    s_d, k_d, v_d = resident_fill_inputs(w, upto=w.seq_lens - 1)
+    fill(k_d, v_d, s_d)
+    main_bulk = bulk_append_report(w, fmt, fill, s_d, k_d, v_d,
+                                   flush=append_bytes(int(s_d.numel()), w.num_kv_heads, fmt)
+                                   < 2 * L2_FLUSH_BYTES)
+    del s_d, k_d, v_d
+    torch.cuda.empty_cache()
+
     # per-step inputs: a few distinct new-token sets, appended at position
     # seq_len - 1 of every sequence
     n_variants = 4
@@ -322,10 +409,7 @@ def run_ours(args):
 
     def append(i):
         j = i % n_variants
-        if fmt == 16:
-            tq.tq_append_bf16(new_k[j], new_v[j], new_slots, cache)
-        else:
-            tq.tq_quantize_append(new_k[j], new_v[j], new_slots, fmt, cache)
+        fill(new_k[j], new_v[j], new_slots)
 
     def dec():
         decode(q, cache, pt, sl, w.q_len, out, max_seq_len=max_len, workspace=ws)
@@ -342,7 +426,7 @@ def run_ours(args):
         tq.tq_hbm_copy(a, bbuf)
         tq.tq_hbm_read(a, sink)
     for _ in range(10):
-        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0, e1, e2 = ev(), ev(), ev()
         e0.record()
         tq.tq_hbm_copy(a, bbuf)
         e1.record()
@@ -357,6 +441,19 @@ def run_ours(args):
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
 
+    # ---- clocks: sampled from here through the timed region; an untimed
+    # soak of about a second first, so the record covers a busy GPU
+    clocks = ClockSampler(local)
+    clocks.start()
+    t_end = time.perf_counter() + 1.0
+    i = 0
+    while time.perf_counter() < t_end:
+        for _ in range(50):
+            append(i)
+            dec()
+            i += 1
+        torch.cuda.synchronize()
+
     # ---- warm-up
     for i in range(args.warmup):
         append(i)
@@ -365,15 +462,12 @@ def run_ours(args):
 
     # ---- timed region (device time, CUDA events on the launching stream)
     K = args.steps
-    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ev_c = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    clocks = ClockSampler(local)
+    ev_a = [ev() for _ in range(K)]
+    ev_b = [ev() for _ in range(K)]
+    ev_c = [ev() for _ in range(K)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)
     for i in range(K):
         ev_a[i].record(stream)
         append(i)
@@ -382,22 +476,30 @@ def run_ours(args):
         ev_c[i].record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
+    if clk is not None:
+        clk["window"] = "about 1 s of untimed steps, the warm-up steps and the timed steps"
     if world > 1:
         dist.barrier()
     total_ms = ev_a[0].elapsed_time(ev_c[-1])
     append_ms = [ev_a[i].elapsed_time(ev_b[i]) for i in range(K)]
     decode_ms = [ev_b[i].elapsed_time(ev_c[i]) for i in range(K)]
 
-    # ---- end to end through the C ABI with host buffers
+    # ---- end to end through the C ABI with host buffers: every step copies
+    # q, the new K/V, their slots, the page table and the lengths from
+    # pinned host memory and reads the output back
     e2e_steps = max(3, min(K, 200))
-    h_q = torch.empty(q.shape, dtype=q.dtype, pin_memory=True).copy_(q.cpu())
-    h_k = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True).copy_(x.cpu()) for x in new_k]
-    h_v = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True).copy_(x.cpu()) for x in new_v]
-    h_s = torch.empty(new_slots.shape, dtype=torch.int64, pin_memory=True).copy_(new_slots.cpu())
+
+    def pinned(t):
+        return torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu())
+
+    h_q, h_s, h_pt, h_sl = pinned(q), pinned(new_slots), pinned(pt), pinned(sl)
+    h_k = [pinned(x) for x in new_k]
+    h_v = [pinned(x) for x in new_v]
     h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     d_q, d_k, d_v, d_s = (torch.empty_like(q), torch.empty_like(new_k[0]),
                           torch.empty_like(new_v[0]), torch.empty_like(new_slots))
-    h2d = (h_q.numel() * 2 + h_k[0].numel() * 2 + h_v[0].numel() * 2 + h_s.numel() * 8)
+    d_pt, d_sl = torch.empty_like(pt), torch.empty_like(sl)
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k[0], h_v[0], h_s, h_pt, h_sl))
     d2h = h_out.numel() * 4
 
     def e2e_step(i):
@@ -406,11 +508,10 @@ def run_ours(args):
         d_k.copy_(h_k[j], non_blocking=True)
         d_v.copy_(h_v[j], non_blocking=True)
         d_s.copy_(h_s, non_blocking=True)
-        if fmt == 16:
-            tq.tq_append_bf16(d_k, d_v, d_s, cache)
-        else:
-            tq.tq_quantize_append(d_k, d_v, d_s, fmt, cache)
-        decode(d_q, cache, pt, sl, w.q_len, out, max_seq_len=max_len, workspace=ws)
+        d_pt.copy_(h_pt, non_blocking=True)
+        d_sl.copy_(h_sl, non_blocking=True)
+        fill(d_k, d_v, d_s)
+        decode(d_q, cache, d_pt, d_sl, w.q_len, out, max_seq_len=max_len, workspace=ws)
         h_out.copy_(out, non_blocking=True)
 
     for i in range(3):
@@ -418,7 +519,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0, e1 = ev(), ev()
     e0.record(stream)
     for i in range(e2e_steps):
         e2e_step(i)
@@ -429,14 +530,14 @@ def run_ours(args):
     err = cache.read_error()
     if err:
         raise SystemExit(f"device error word set: 0x{err:x}")
+    del cache, ws, q, pt, sl, out, new_k, new_v
+    torch.cuda.empty_cache()
 
     # ---- reduce over ranks: max of each time
     ms_step, dec_avg, app_avg, e2e_ms = max_over_ranks(
         [total_ms / K, sum(decode_ms) / K, sum(append_ms) / K, e2e_ms], world, dev)
 
     kv_bytes, app_bytes = step_bytes(w, fmt)
-    peaks, peak_kind = measured_peaks()
-    peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     value = job_throughput(kv_bytes, world, ms_step)
     achieved = kv_bytes / (dec_avg * 1e-3) / 1e9
     line = {
@@ -450,12 +551,15 @@ def run_ours(args):
         "seq_per_s": world * w.batch / (ms_step * 1e-3),
         "decode_kv_gbs": achieved,
         "decode_ms": dec_avg,
+        "decode_kernel": decode_kernel_label(fmt, w.q_len * w.group),
         "append_gbs": app_bytes / (app_avg * 1e-3) / 1e9,
         "append_ms": app_avg,
+        "append_bulk": main_bulk,
         "hbm_inrun_gbs": {"copy": copy_gbs, "read": read_gbs},
         "frac_of_hbm": {"step": (value / world) / peak, "decode_kernel": achieved / peak,
                         "decode_vs_inrun_copy": achieved / copy_gbs,
-                        "decode_vs_inrun_read": achieved / read_gbs},
+                        "decode_vs_inrun_read": achieved / read_gbs,
+                        "append_bulk": main_bulk["frac_of_hbm"]},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": profiled_traffic("decode"),
                      "peak_source": f"hbm_gbs of {peak_kind}",
@@ -465,6 +569,11 @@ def run_ours(args):
         "gpu_launches": 2 * K,
         "clocks": clk,
     }
+
+    # ================================================== every configuration
+    if not args.no_per_config:
+        line["per_config"] = per_config(tq, dev, peak, resident_fill_inputs, appender, timed,
+                                        bulk_append_report)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, fmt)
     if world > 1:
@@ -473,6 +582,66 @@ def run_ours(args):
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def per_config(tq, dev, peak, resident_fill_inputs, appender, timed, bulk_append_report):
+    """Decode (and bulk append) of every synthetic workload and format, each
+    alone on the GPU with inputs resident and the L2 flushed before every
+    timed launch: decode us, KV GB/s, seq/s (tokens/s for verify windows) and
+    fractions of the HBM peak; for shared prefixes also the fraction counted
+    on unique bytes."""
+    import torch
+    rows = []
+    for name in dict.fromkeys(n for n, _ in PER_CONFIG):
+        w = W.make(name)
+        s_d, k_d, v_d = resident_fill_inputs(w)
+        q = torch.from_numpy(w.queries().view(np.int16)).view(torch.bfloat16).to(dev)
+        pt = torch.from_numpy(w.page_table).to(dev)
+        sl = torch.from_numpy(w.seq_lens).to(dev)
+        out = torch.empty((w.batch, w.q_len, w.num_q_heads, w.head_dim), dtype=torch.float32,
+                          device=dev)
+        for nm, fmt in PER_CONFIG:
+            if nm != name:
+                continue
+            cache = tq.Cache(fmt, w.num_pages, w.num_kv_heads, w.page_size, device=dev)
+            fill = appender(cache, fmt)
+            fill(k_d, v_d, s_d)
+            bulk = bulk_append_report(w, fmt, fill, s_d, k_d, v_d, flush=True)
+            ws = cache.workspace(w.batch, w.q_len, w.num_q_heads, w.max_seq_len)
+            fn = tq.tq_paged_decode_bf16 if fmt == 16 else tq.tq_paged_decode
+
+            def dec():
+                fn(q, cache, pt, sl, w.q_len, out, max_seq_len=w.max_seq_len, workspace=ws)
+
+            for _ in range(3):
+                dec()
+            ms, ms_min = timed(dec, 20, flush=True)
+            err = cache.read_error()
+            if err:
+                raise SystemExit(f"{name}/{fmt}: device error word set: 0x{err:x}")
+            kv = w.tokens_read() * 2 * W.row_bytes(fmt)
+            gbs = kv / (ms * 1e-3) / 1e9
+            r = {"workload": name, "format": FORMAT_NAMES[fmt],
+                 "kernel": decode_kernel_label(fmt, w.q_len * w.group),
+                 "batch": w.batch, "q_len": w.q_len, "q_heads": w.num_q_heads,
+                 "kv_heads": w.num_kv_heads, "page_size": w.page_size,
+                 "tokens": int(w.seq_lens.sum()),
+                 "decode_us": ms * 1e3, "decode_us_min": ms_min * 1e3,
+                 "kv_bytes": kv, "kv_gbs": gbs, "frac_of_hbm": gbs / peak,
+                 "seq_per_s": w.batch / (ms * 1e-3), "append_bulk": bulk,
+                 "l2": "flushed before every timed launch"}
+            if w.q_len > 1:
+                r["tokens_per_s"] = w.batch * w.q_len / (ms * 1e-3)
+            uniq = w.unique_tokens_read() * 2 * W.row_bytes(fmt)
+            if uniq != kv:
+                r["unique_kv_bytes"] = uniq
+                r["unique_frac_of_hbm"] = uniq / (ms * 1e-3) / 1e9 / peak
+            rows.append(r)
+            del cache, ws
+            torch.cuda.empty_cache()
+        del s_d, k_d, v_d, q, pt, sl, out
+        torch.cuda.empty_cache()
+    return rows
 
 
 def main(argv=None):
@@ -484,6 +653,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=W.ALL)
     ap.add_argument("--fmt", type=int, default=0, help="cache format (default: workload's first)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per-configuration decode and bulk-append timings")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
