@@ -32,7 +32,8 @@ _LIB = os.path.join(_HERE, "libtq_oracle.so")
 CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
           "-fPIC", "-shared", "-Wall", "-Wextra"]
 
-FORMAT_BITS = {2: 2, 3: 3, 4: 4, 8: 8, 16: 0}
+FORMAT_BITS = {2: 2, 3: 3, 4: 4, 8: 8, 16: 0, 17: 8}
+FP8 = 17          # the fp8 (E4M3) format id
 
 
 def build(force: bool = False) -> str:
@@ -78,6 +79,12 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_paged_decode.restype = I
         _lib.oracle_attention_f64.argtypes = [P, P, P, I, I, I, P]
         _lib.oracle_attention_f64.restype = None
+        _lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        _lib.oracle_e4m3_value.restype = ctypes.c_double
+        _lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        _lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        _lib.oracle_fp8_quantize_vector.argtypes = [P, I, P, P]
+        _lib.oracle_fp8_quantize_vector.restype = None
     return _lib
 
 
@@ -149,9 +156,27 @@ def quantize_vector(x_bf16, bits: int):
     return out, s[0]
 
 
+def e4m3_value(code: int) -> float:
+    return float(lib().oracle_e4m3_value(code))
+
+
+def e4m3_encode(y: float) -> int:
+    return int(lib().oracle_e4m3_encode(y))
+
+
+def fp8_quantize_vector(x_bf16):
+    """(E4M3 code bytes, fp32 scale) of one bf16 head vector (no rotation)."""
+    x = _c(x_bf16, np.uint16)
+    out = np.empty(x.shape[-1], np.uint8)
+    s = np.zeros(1, np.float32)
+    lib().oracle_fp8_quantize_vector(_ptr(x), x.shape[-1], _ptr(out), _ptr(s))
+    return out, s[0]
+
+
 def quantize_append(k_bf16, v_bf16, slot_mapping, bits: int, page_size: int,
                     k_pages: np.ndarray, v_pages: np.ndarray) -> None:
-    """Append into uint8 page pools shaped [num_pages][num_kv_heads][block]."""
+    """Append into uint8 page pools shaped [num_pages][num_kv_heads][block];
+    `bits` is the format: 2, 3, 4, 8 (turbo) or FP8 (17)."""
     k = _c(k_bf16, np.uint16)
     v = _c(v_bf16, np.uint16)
     slots = _c(slot_mapping, np.int64)

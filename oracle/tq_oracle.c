@@ -35,6 +35,18 @@
  *   causality  query position t of q_len sees keys j <= seq_len - q_len + t.
  *   GQA        query head h reads kv head h / (num_q_heads / num_kv_heads).
  *
+ * fp8 (format 17, the --kvcache-dtype fp8 choice of the xInfer page; the
+ * pages give only "fp8", "2x" and "near-lossless", this oracle fixes it):
+ *   codes      OCP E4M3 (1 sign, 4 exponent bits of bias 7, 3 mantissa bits,
+ *              no infinities, largest finite 448); no rotation.
+ *   scale      s = max_i |x_i| (fp32), stored as fp32; s == 0 gives codes 0.
+ *   codes      y_i = fl(fl(x_i * 448) / s) (IEEE fp32), code_i = the E4M3
+ *              value nearest y_i, ties to the even code, |y_i| > 448 to 448.
+ *   storage    one byte per code (the E4M3 bit pattern), in the block layout
+ *              of turbo8.
+ *   dequant    xhat_i = value(code_i) * s / 448 in fp64; attention as for
+ *              BF16 (no rotation) on the dequantised K and V.
+ *
  * Cache layout (an interface, described in include/tq.h, implemented here
  * independently): blocks are ordered [page][kv_head].  For a turbo format
  * with b bits and page size P, a K block holds P token rows of d*b/8 code
@@ -61,14 +73,66 @@ static float bf16_to_f32(uint16_t bits)
     return f;
 }
 
-/* number of code bits of a turbo format, 0 for bf16, -1 if unknown */
+enum { FORMAT_FP8 = 17 };
+
+/* number of code bits of a turbo or fp8 format, 0 for bf16, -1 if unknown */
 static int format_bits(int format)
 {
     switch (format) {
     case 2: case 3: case 4: case 8: return format;
+    case FORMAT_FP8: return 8;
     case 16: return 0;
     default: return -1;
     }
+}
+
+/* Value of an E4M3 code (OCP "e4m3fn": 0x7F and 0xFF are NaN). */
+ORACLE_API double oracle_e4m3_value(uint8_t c)
+{
+    const int e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return NAN;
+    const double v = e == 0 ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return (c & 0x80) ? -v : v;
+}
+
+/* The E4M3 code nearest y, found by comparing y with every finite
+ * non-negative code; a tie goes to the code with an even mantissa; |y|
+ * above the largest finite value (448) gives 448.  The sign of y is kept
+ * (-0 gives 0x80). */
+ORACLE_API uint8_t oracle_e4m3_encode(float y)
+{
+    const uint8_t sgn = signbit(y) ? 0x80 : 0x00;
+    const double a = fabs((double)y);
+    int best = 0;
+    double best_d = a;                          /* code 0: value 0 */
+    for (int c = 1; c <= 0x7E; ++c) {
+        const double dd = fabs(a - oracle_e4m3_value((uint8_t)c));
+        if (dd < best_d || (dd == best_d && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_d = dd;
+        }
+    }
+    return (uint8_t)(sgn | best);
+}
+
+/* fp8 codes and scale of one bf16 head vector (no rotation). */
+ORACLE_API void oracle_fp8_quantize_vector(const uint16_t* x_bf16, int d, uint8_t* codes,
+                                           float* scale)
+{
+    float s = 0.0f;
+    for (int i = 0; i < d; ++i) {
+        float a = fabsf(bf16_to_f32(x_bf16[i]));
+        if (a > s) s = a;
+    }
+    for (int i = 0; i < d; ++i) {
+        if (s == 0.0f) {
+            codes[i] = 0;
+            continue;
+        }
+        float t = bf16_to_f32(x_bf16[i]) * 448.0f;
+        codes[i] = oracle_e4m3_encode(t / s);
+    }
+    *scale = s;
 }
 
 static int64_t oracle_block_bytes_impl(int format, int d, int page_size)
@@ -215,12 +279,14 @@ ORACLE_API void oracle_quantize_vector(const uint16_t* x_bf16, int d, int bits,
 ORACLE_API int oracle_quantize_append(const uint16_t* k, const uint16_t* v,
                                       const int64_t* slot_mapping,
                                       int num_tokens, int num_kv_heads, int d,
-                                      int bits, int page_size, int num_pages,
+                                      int format, int page_size, int num_pages,
                                       uint8_t* k_pages, uint8_t* v_pages)
 {
-    if (format_bits(bits) <= 0) return OR_BAD_ARG;
-    int64_t bb = oracle_block_bytes_impl(bits, d, page_size);
+    if (format_bits(format) <= 0) return OR_BAD_ARG;
+    int64_t bb = oracle_block_bytes_impl(format, d, page_size);
     if (bb < 0) return OR_BAD_ARG;
+    const int bits = format_bits(format);
+    const int fp8 = format == FORMAT_FP8;
     const int cb = d * bits / 8;
     float* y = (float*)malloc(sizeof(float) * (size_t)d);
     int32_t* codes = (int32_t*)malloc(sizeof(int32_t) * (size_t)d);
@@ -236,15 +302,25 @@ ORACLE_API int oracle_quantize_append(const uint16_t* k, const uint16_t* v,
             const uint16_t* kx = k + ((size_t)t * num_kv_heads + h) * d;
             const uint16_t* vx = v + ((size_t)t * num_kv_heads + h) * d;
             float ks, vs;
-            /* K: the token's packed vector is row `off` of the block */
-            oracle_quantize_vector(kx, d, bits, k_pages + blk + off * cb, &ks);
-            /* V: code i goes to row i (dim-major), field `off` */
-            oracle_rotate_f32(vx, d, y);
-            oracle_quantize_rotated(y, d, bits, codes, &vs);
-            const int L = (1 << (bits - 1)) - 1;
-            for (int i = 0; i < d; ++i)
-                put_bits(v_pages + blk, (int64_t)i * page_size * bits + (int64_t)off * bits,
-                         bits, (uint32_t)(codes[i] + L));
+            if (fp8) {
+                /* K: row `off` holds the token's d code bytes; V: byte `off`
+                   of dimension row i holds code i */
+                oracle_fp8_quantize_vector(kx, d, k_pages + blk + off * cb, &ks);
+                uint8_t* vc = (uint8_t*)malloc((size_t)d);
+                oracle_fp8_quantize_vector(vx, d, vc, &vs);
+                for (int i = 0; i < d; ++i) v_pages[blk + (size_t)i * page_size + off] = vc[i];
+                free(vc);
+            } else {
+                /* K: the token's packed vector is row `off` of the block */
+                oracle_quantize_vector(kx, d, bits, k_pages + blk + off * cb, &ks);
+                /* V: code i goes to row i (dim-major), field `off` */
+                oracle_rotate_f32(vx, d, y);
+                oracle_quantize_rotated(y, d, bits, codes, &vs);
+                const int L = (1 << (bits - 1)) - 1;
+                for (int i = 0; i < d; ++i)
+                    put_bits(v_pages + blk, (int64_t)i * page_size * bits + (int64_t)off * bits,
+                             bits, (uint32_t)(codes[i] + L));
+            }
             memcpy(k_pages + blk + (size_t)page_size * cb + off * 4, &ks, 4);
             memcpy(v_pages + blk + (size_t)page_size * cb + off * 4, &vs, 4);
         }
@@ -280,13 +356,20 @@ ORACLE_API int oracle_append_bf16(const uint16_t* k, const uint16_t* v,
  * dim_major selects the V block layout (dimension rows of token fields). */
 static void dequant_token(const uint8_t* pages, int64_t bb, int page, int kvh,
                           int num_kv_heads, int off, int page_size, int d,
-                          int bits, int dim_major, int32_t* codes, double* out)
+                          int bits, int dim_major, int fp8, int32_t* codes, double* out)
 {
     const int L = (1 << (bits - 1)) - 1;
     const int cb = d * bits / 8;
     const uint8_t* blk = pages + (size_t)(((int64_t)page * num_kv_heads + kvh) * bb);
     float s;
     memcpy(&s, blk + (size_t)page_size * cb + (size_t)off * 4, 4);
+    if (fp8) {
+        for (int i = 0; i < d; ++i) {
+            const uint8_t c = dim_major ? blk[(size_t)i * page_size + off] : blk[(size_t)off * cb + i];
+            out[i] = oracle_e4m3_value(c) * (double)s / 448.0;
+        }
+        return;
+    }
     if (dim_major) {
         for (int i = 0; i < d; ++i)
             codes[i] = (int32_t)get_bits(blk, (int64_t)i * page_size * bits +
@@ -413,10 +496,10 @@ ORACLE_API int oracle_paged_decode(const uint16_t* q, int format, int d,
                     if (bits > 0) {
                         dequant_token((const uint8_t*)k_pages, bb, page, kvh,
                                       num_kv_heads, j % page_size, page_size, d,
-                                      bits, 0, codes, kr);
+                                      bits, 0, format == FORMAT_FP8, codes, kr);
                         dequant_token((const uint8_t*)v_pages, bb, page, kvh,
                                       num_kv_heads, j % page_size, page_size, d,
-                                      bits, 1, codes, vr);
+                                      bits, 1, format == FORMAT_FP8, codes, vr);
                     } else {
                         bf16_token((const uint16_t*)k_pages, page, kvh,
                                    num_kv_heads, j % page_size, page_size, d, kr);
@@ -428,7 +511,8 @@ ORACLE_API int oracle_paged_decode(const uint16_t* q, int format, int d,
                 const uint16_t* qb = q + (((size_t)b * q_len + t) * num_q_heads + h) * d;
                 for (int i = 0; i < d; ++i) qx[i] = (double)bf16_to_f32(qb[i]);
                 double* dst = out + (((size_t)b * q_len + t) * num_q_heads + h) * d;
-                oracle_attention_f64(qx, K, V, visible, d, bits > 0, dst);
+                /* turbo formats attend in the rotated basis; fp8 and bf16 do not */
+                oracle_attention_f64(qx, K, V, visible, d, bits > 0 && format != FORMAT_FP8, dst);
             }
         }
     }

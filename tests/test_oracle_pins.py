@@ -469,3 +469,152 @@ def test_quantize_append_layout_and_skip(bits, P):
                 assert not kp[page, :, off * cb:(off + 1) * cb].any()
                 for h in range(2):
                     assert not _unpack_u(vp, bits, page, h, off, P, True).any()
+
+
+# ----------------------------------------------------------------- fp8
+FP8 = oracle.FP8
+
+
+def test_e4m3_values_match_torch_float8():
+    """Every E4M3 code's value equals torch's float8_e4m3fn (a library
+    routine), NaN codes included."""
+    codes = torch.arange(256, dtype=torch.uint8)
+    lib_vals = codes.view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    ours = np.array([oracle.e4m3_value(c) for c in range(256)])
+    assert np.array_equal(np.isnan(lib_vals), np.isnan(ours))
+    ok = ~np.isnan(ours)
+    assert np.array_equal(lib_vals[ok], ours[ok])
+    assert oracle.e4m3_value(0x7E) == 448.0 and oracle.e4m3_value(0x01) == 2.0 ** -9
+
+
+def test_e4m3_rounding_golden():
+    for v_hex, c_hex in read_golden("e4m3_rounding.txt"):
+        v = np.uint32(int(v_hex, 16)).view(np.float32)
+        assert oracle.e4m3_encode(float(v)) == int(c_hex, 16), v_hex
+
+
+def test_e4m3_encode_matches_torch_cast():
+    """Round to nearest, ties to even, saturating below the NaN midpoint:
+    the same codes as torch's fp32 -> float8_e4m3fn cast on values spread
+    over every binade and the subnormals."""
+    rng = np.random.default_rng(60)
+    x = rng.standard_normal(20000) * 10.0 ** rng.uniform(-4.5, 2.6, 20000)
+    x = np.clip(x, -460.0, 460.0).astype(np.float32)
+    lib_codes = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    ours = np.array([oracle.e4m3_encode(float(v)) for v in x], np.uint8)
+    assert np.array_equal(lib_codes, ours)
+
+
+def test_fp8_quantizer_closed_forms():
+    """x = a e_j: s = |a| and y_j = fl(fl(a 448) / |a|) = +-448 exactly, so
+    code j is 0x7E or 0xFE and every other code is +0; x = 0 gives s = 0 and
+    codes 0."""
+    for a, j in ((1.0, 0), (-3.5, 7), (0.0078125, 127)):
+        x = np.zeros(128, np.float32)
+        x[j] = a
+        codes, s = oracle.fp8_quantize_vector(W.f32_to_bf16_bits(x))
+        assert s == abs(a)
+        assert codes[j] == (0x7E if a > 0 else 0xFE)
+        assert np.all(np.delete(codes, j) == 0)
+    codes, s = oracle.fp8_quantize_vector(np.zeros(128, np.uint16))
+    assert s == 0 and not codes.any()
+
+
+def test_fp8_pow2_equivariance_and_error_bound():
+    """x 2^k keeps every code (bit-exact) and scales s by 2^k; the
+    dequantised value is within half an E4M3 step of x: |xhat - x| <=
+    s/448 * max(|y| 2^-4, 2^-10) (plus fp32 slack)."""
+    rng = np.random.default_rng(61)
+    for _ in range(100):
+        xb = rand_bf16(rng, 128, scale=rng.uniform(0.01, 50))
+        c0, s0 = oracle.fp8_quantize_vector(xb)
+        for k in (-4, 3):
+            xk = W.f32_to_bf16_bits(W.bf16_bits_to_f32(xb) * np.float32(2.0 ** k))
+            ck, sk = oracle.fp8_quantize_vector(xk)
+            assert np.array_equal(c0, ck) and sk == np.float32(s0 * np.float32(2.0 ** k))
+        x = W.bf16_bits_to_f32(xb).astype(np.float64)
+        xhat = np.array([oracle.e4m3_value(c) for c in c0]) * float(s0) / 448.0
+        y = np.abs(x) * 448.0 / float(s0)
+        bound = float(s0) / 448.0 * np.maximum(y * 2.0 ** -4, 2.0 ** -10) * (1 + 2.0 ** -20)
+        assert np.all(np.abs(xhat - x) <= bound + 1e-30)
+        assert np.max(np.abs(xhat)) == float(s0)          # the absmax element is exact
+
+
+def test_fp8_append_layout():
+    """fp8 blocks have turbo8's layout: K token rows of 128 code bytes, V
+    dimension rows of page_size code bytes, fp32 scales after the codes."""
+    rng = np.random.default_rng(62)
+    P = 16
+    k = rand_bf16(rng, (3, 2, 128))
+    v = rand_bf16(rng, (3, 2, 128))
+    bb = oracle.block_bytes(FP8, 128, P)
+    assert bb == P * 132
+    kp = np.zeros((2, 2, bb), np.uint8)
+    vp = np.zeros_like(kp)
+    slots = np.array([3, -1, P + 15])
+    oracle.quantize_append(k, v, slots, FP8, P, kp, vp)
+    for t, (page, off) in ((0, (0, 3)), (2, (1, 15))):
+        for h in range(2):
+            ck, sk = oracle.fp8_quantize_vector(k[t, h])
+            cv, sv = oracle.fp8_quantize_vector(v[t, h])
+            assert np.array_equal(kp[page, h, off * 128:(off + 1) * 128], ck)
+            assert np.array_equal(vp[page, h, :P * 128].reshape(128, P)[:, off], cv)
+            assert kp[page, h, P * 128 + 4 * off:P * 128 + 4 * off + 4].view(np.float32)[0] == sk
+            assert vp[page, h, P * 128 + 4 * off:P * 128 + 4 * off + 4].view(np.float32)[0] == sv
+
+
+@pytest.mark.parametrize("q_len", [1, 3])
+def test_fp8_paged_decode_matches_sdpa(q_len):
+    """fp8 decode is plain softmax attention (no rotation) on the
+    dequantised K and V: torch SDPA in fp64 on the same values."""
+    w = W.custom(batch=2, num_q_heads=4, num_kv_heads=2, page_size=16, q_len=q_len,
+                 seq_lens=(45, 17 + q_len), fmt=FP8, seed=63)
+    kp, vp = _pools(w, FP8)
+    for slots, k, v in w.iter_fill():
+        oracle.quantize_append(k, v, slots, FP8, w.page_size, kp, vp)
+    q = w.queries()
+    out = oracle.paged_decode(q, FP8, w.page_size, kp, vp, w.page_table, w.seq_lens,
+                              w.num_kv_heads)
+    P = w.page_size
+    for b in range(w.batch):
+        n = int(w.seq_lens[b])
+        for h in range(w.num_q_heads):
+            kvh = h // w.group
+            K = np.zeros((n, 128))
+            V = np.zeros((n, 128))
+            for j in range(n):
+                page, off = int(w.page_table[b, j // P]), j % P
+                blk_k, blk_v = kp[page, kvh], vp[page, kvh]
+                sk = blk_k[P * 128 + 4 * off:P * 128 + 4 * off + 4].view(np.float32)[0]
+                sv = blk_v[P * 128 + 4 * off:P * 128 + 4 * off + 4].view(np.float32)[0]
+                K[j] = torch.from_numpy(blk_k[off * 128:(off + 1) * 128].copy()).view(
+                    torch.float8_e4m3fn).double().numpy() * float(sk) / 448.0
+                V[j] = torch.from_numpy(blk_v[:P * 128].reshape(128, P)[:, off].copy()).view(
+                    torch.float8_e4m3fn).double().numpy() * float(sv) / 448.0
+            qr = W.bf16_bits_to_f32(q[b, :, h]).astype(np.float64)
+            ref = _sdpa(qr, K, V, [n - q_len + t for t in range(q_len)])
+            assert np.max(np.abs(out[b, :, h] - ref)) < 1e-11
+
+
+def test_fp8_division_order_golden():
+    """fl(fl(x 448) / s): on each row the exact quotient is an E4M3
+    midpoint reached exactly, so the code is the even neighbour; the
+    reciprocal multiply (rows 1-3) or the late multiply (rows 4-6) would
+    give the odd one."""
+    from fractions import Fraction
+    for x_hex, s_hex, code_s, other_s in read_golden("fp8_division_order.txt"):
+        x = np.uint32(int(x_hex, 16)).view(np.float32)
+        s = np.uint32(int(s_hex, 16)).view(np.float32)
+        X, S = Fraction(float(x)), Fraction(float(s))
+        y = _fl32(_fl32(X * 448) / S)
+        assert y == X * 448 / S                        # both steps exact: the midpoint itself
+        lo_hi = sorted(oracle.e4m3_value(c) for c in (int(code_s, 16), int(other_s, 16)))
+        assert y == (Fraction(lo_hi[0]) + Fraction(lo_hi[1])) / 2
+        assert int(code_s, 16) % 2 == 0 and int(other_s, 16) % 2 == 1
+        vec = np.zeros(128, np.float32)
+        vec[0], vec[1] = s, x
+        codes, scale = oracle.fp8_quantize_vector(W.f32_to_bf16_bits(vec))
+        assert scale == s and codes[0] == 0x7E and codes[1] == int(code_s, 16)
+        recip = oracle.e4m3_encode(float(_fl32(X * _fl32(Fraction(448) / S))))
+        late = oracle.e4m3_encode(float(_fl32(_fl32(X / S) * 448)))
+        assert int(other_s, 16) in (recip, late)
