@@ -97,12 +97,15 @@ ORACLE_API double oracle_e4m3_value(uint8_t c)
 
 /* The E4M3 code nearest y, found by comparing y with every finite
  * non-negative code; a tie goes to the code with an even mantissa; |y|
- * above the largest finite value (448) gives 448.  The sign of y is kept
+ * above the largest finite value (448), infinity included, gives 448 (the
+ * format saturates); NaN gives the NaN code 0x7F.  The sign of y is kept
  * (-0 gives 0x80). */
 ORACLE_API uint8_t oracle_e4m3_encode(float y)
 {
     const uint8_t sgn = signbit(y) ? 0x80 : 0x00;
     const double a = fabs((double)y);
+    if (isnan(a)) return (uint8_t)(sgn | 0x7F);
+    if (a > 448.0) return (uint8_t)(sgn | 0x7E);   /* every finite code is nearer than inf */
     int best = 0;
     double best_d = a;                          /* code 0: value 0 */
     for (int c = 1; c <= 0x7E; ++c) {
