@@ -66,7 +66,7 @@ def job_throughput(bytes_per_rank_step: int, world: int, ms_step: float) -> floa
 
 
 def describe(w: W.Workload, fmt: int) -> str:
-    names = {2: "turbo2", 3: "turbo3", 4: "turbo4", 8: "turbo8", 16: "bf16"}
+    names = FORMAT_NAMES
     lens = (f"{int(w.seq_lens[0])} tokens" if np.all(w.seq_lens == w.seq_lens[0])
             else f"lengths {int(w.seq_lens.min())}-{int(w.seq_lens.max())}")
     return (f"{w.name}: batch {w.batch} x {lens}, {w.num_q_heads} q / {w.num_kv_heads} kv "
@@ -268,8 +268,8 @@ def run_reference(args):
 # The (workload, format) pairs timed in `per_config`: every format of every
 # synthetic workload (the bench workload itself is the line's main part).
 PER_CONFIG = (("tiny", 4), ("batch8", 4), ("cbatch64", 3), ("cbatch64", 8), ("cbatch64", 16),
-              ("long128k", 4), ("long128k", 2), ("specverify", 4))
-FORMAT_NAMES = {2: "turbo2", 3: "turbo3", 4: "turbo4", 8: "turbo8", 16: "bf16"}
+              ("cbatch64", 17), ("long128k", 4), ("long128k", 2), ("specverify", 4))
+FORMAT_NAMES = {2: "turbo2", 3: "turbo3", 4: "turbo4", 8: "turbo8", 16: "bf16", 17: "fp8"}
 L2_FLUSH_BYTES = 256 << 20         # > the 126 MB L2
 
 
@@ -279,6 +279,8 @@ def decode_kernel_label(fmt: int, G: int) -> str:
     if fmt == 16:
         return "k_decode<16>"
     rows = 4 if G <= 4 else (8 if G <= 8 else 16)
+    if fmt == 17:
+        return f"k_decode_tc<8,{rows},fp8>"
     if fmt == 3 or rows == 16:
         return f"k_decode_tc<{fmt},{rows}>"
     return f"k_decode_i8<{fmt},{rows}>"

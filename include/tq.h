@@ -23,6 +23,14 @@
  *             yhat_k,j / sqrt(d); out = H (sum_j softmax_j yhat_v,j) / sqrt(d).
  *             Query position t of q_len sees keys j <= seq_len - q_len + t.
  *             Query head h reads kv head h / (num_q_heads / num_kv_heads).
+ *   fp8       (--kvcache-dtype fp8 of "Getting a server up"; 2x, "near-
+ *             lossless" in "TurboQuant is a memory trade"; the rest is this
+ *             library's reading) no rotation; s = max_i |x_i| as fp32; code_i
+ *             = the OCP E4M3 value nearest fl(fl(x_i * 448) / s), ties to the
+ *             even mantissa, saturating at 448 (s == 0: codes 0), stored as its
+ *             byte; dequantised xhat_i = value(code_i) * s / 448; attention
+ *             softmax(q . k / sqrt(d)) v on the dequantised K and V.  Its
+ *             blocks have the turbo8 layout below.
  *
  * Cache layout in device memory (one pool per layer):
  *   pool[num_pages][num_kv_heads][2][block], block = tq_page_block_bytes(...):
@@ -70,7 +78,7 @@
 extern "C" {
 #endif
 
-#define TQ_ABI_VERSION 2
+#define TQ_ABI_VERSION 3
 
 typedef enum {
     TQ_OK = 0,
@@ -79,7 +87,8 @@ typedef enum {
     TQ_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
     TQ_ERR_TIMEOUT = 4,       /* a bounded device wait expired (device word) */
     TQ_ERR_DEVICE_CHECK = 5,  /* a device-side range check failed (device word) */
-    TQ_ERR_WORKSPACE = 6      /* decode workspace missing or too small */
+    TQ_ERR_WORKSPACE = 6,     /* decode workspace missing or too small */
+    TQ_ERR_NO_PAGES = 7       /* prefix-block manager: the pool has no page left */
 } tq_status;
 
 /* KV cache formats: the --kvcache-dtype choices of the xInfer page (section
@@ -89,7 +98,8 @@ typedef enum {
     TQ_TURBO3 = 3,
     TQ_TURBO4 = 4,
     TQ_TURBO8 = 8,
-    TQ_BF16 = 16
+    TQ_BF16 = 16,
+    TQ_FP8 = 17      /* E4M3 codes, no rotation (see "fp8" above) */
 } tq_format;
 
 /* Descriptor of one layer's paged K/V pool.  Plain data; the pointed-to
@@ -252,6 +262,124 @@ tq_status tq_read_device_error(const tq_cache* cache, uint32_t* code,
 tq_status tq_hbm_copy(const void* src, void* dst, size_t bytes, void* stream);
 tq_status tq_hbm_read(const void* src, size_t bytes, uint32_t* sink,
                       void* stream);
+
+/*
+ * One decode step captured as a CUDA graph: "CUDA Graphs mean the decode step
+ * is captured as a graph and replayed, which removes per-token launch
+ * overhead" (xInfer review, "What actually sits between the request and the
+ * tokens").  The step is the append of num_tokens new tokens (skipped when 0;
+ * tq_quantize_append for a turbo cache, tq_append_bf16 for a BF16 one)
+ * followed by the paged decode (skipped when batch is 0), with exactly the
+ * arguments of those calls.  Every pointer and size is fixed at capture: the
+ * caller refreshes the contents of the buffers (new K/V, slots, q, page
+ * table, lengths) between launches, keeping q_len, batch and max_seq_len.
+ * The decode workspace returns its counters to zero after every step, so a
+ * graph can be replayed any number of times.
+ */
+typedef struct {
+    const void* k;                  /* append: as tq_quantize_append */
+    const void* v;
+    const int64_t* slot_mapping;
+    int32_t num_tokens;
+    const void* q;                  /* decode: as tq_paged_decode */
+    const int32_t* page_table;
+    int32_t max_pages_per_seq;
+    const int32_t* seq_lens;
+    int32_t batch;
+    int32_t q_len;
+    int32_t num_q_heads;
+    int32_t max_seq_len;
+    float* out;
+    void* workspace;
+    size_t workspace_bytes;
+} tq_step;
+
+typedef struct tq_step_graph tq_step_graph;
+
+/* Validate the step as the two calls would, then capture it on `stream` (a
+ * created stream, not NULL: the legacy stream cannot be captured) and
+ * instantiate it.  Nothing runs on the GPU.  *graph is NULL on failure. */
+tq_status tq_step_graph_create(const tq_cache* cache, const tq_step* step, void* stream,
+                               tq_step_graph** graph);
+/* Run the captured step on `stream` (asynchronous). */
+tq_status tq_step_graph_launch(tq_step_graph* graph, void* stream);
+void tq_step_graph_destroy(tq_step_graph* graph);
+
+/*
+ * Prefix-block manager -- block-granular KV reuse across requests, host side.
+ * "xinfer-ai" package docs, "Prefix Cache (KV Reuse)": finished sequences give
+ * their full KV blocks to a global prefix cache; a new request reuses the
+ * longest cached block-aligned prefix and prefills only the rest; a common
+ * prefix ending inside a block has that block's tail recomputed; a prompt
+ * cached entirely at block boundaries recomputes its last block (the prefill
+ * step is never empty); the cache shares the pool with live sequences and is
+ * capped at a token count rounded down to whole blocks.
+ *
+ * A block is one page of page_size tokens.  The manager hands out page ids of
+ * a pool of num_pages pages (the pool itself is the caller's device memory,
+ * described by a tq_cache with the same page_size and num_pages); a cached
+ * page is shared by every sequence whose prompt starts with the same blocks
+ * of token ids.  Pages are reference counted (one reference per live
+ * sequence holding the page, one while it is cached); when no page is free,
+ * or the cache is over its cap, the least recently used cached block that no
+ * live sequence holds and that has no cached children is evicted.  All calls
+ * are host-only (no device memory is touched) and thread-safe; the caller
+ * copies the page tables to the device.  Errors: TQ_ERR_INVALID_ARG for bad
+ * arguments, TQ_ERR_NO_PAGES when the pool cannot supply the pages (nothing
+ * changes then).
+ */
+typedef struct tq_prefix_cache tq_prefix_cache;
+
+typedef struct {
+    int64_t free_pages;       /* pages no sequence or cached block holds */
+    int64_t cached_blocks;    /* blocks in the prefix cache */
+    int64_t live_sequences;   /* begun and not finished */
+    int64_t hit_tokens;       /* prompt tokens served from the cache, summed over calls */
+    int64_t prompt_tokens;    /* prompt tokens admitted, summed over calls */
+    int64_t evictions;        /* cached blocks evicted */
+} tq_prefix_stats;
+
+/* A manager for num_pages pages of page_size tokens; at most
+ * max_cached_tokens / page_size blocks stay cached (<= 0: half the pool).
+ * NULL for bad arguments or when host memory runs out. */
+tq_prefix_cache* tq_prefix_cache_create(int32_t num_pages, int32_t page_size,
+                                        int64_t max_cached_tokens);
+void tq_prefix_cache_destroy(tq_prefix_cache* pc);
+
+/*
+ * tq_prefix_cache_begin -- admit a sequence whose prompt is the token ids
+ * tokens[0 .. num_tokens), num_tokens >= 1.
+ *   page_table     host int32 [max_pages]: entries [0, ceil(num_tokens /
+ *                  page_size)) are written -- the shared pages of the reused
+ *                  prefix blocks, then fresh pages.
+ *   cached_tokens  the prompt tokens whose K/V the pool holds already (a
+ *                  multiple of page_size): append tokens [cached_tokens,
+ *                  num_tokens) before decoding.
+ *   seq            a handle for tq_prefix_cache_extend / _finish.
+ */
+tq_status tq_prefix_cache_begin(tq_prefix_cache* pc, const int32_t* tokens, int32_t num_tokens,
+                                int32_t* page_table, int32_t max_pages,
+                                int32_t* cached_tokens, int32_t* seq);
+
+/* Grow sequence seq to new_len tokens: fresh pages are added at the end of
+ * its table and the whole table is written to page_table (host int32
+ * [max_pages]). */
+tq_status tq_prefix_cache_extend(tq_prefix_cache* pc, int32_t seq, int32_t new_len,
+                                 int32_t* page_table, int32_t max_pages);
+
+/* Finish sequence seq, whose token ids (prompt and generated) are
+ * tokens[0 .. num_tokens): each of its full blocks joins the cache (a block
+ * already cached keeps its cached page and this sequence's copy is freed),
+ * the rest of its pages are freed, and the cache is trimmed to its cap.
+ * The handle is invalid afterwards. */
+tq_status tq_prefix_cache_finish(tq_prefix_cache* pc, int32_t seq, const int32_t* tokens,
+                                 int32_t num_tokens);
+
+/* Counters of the manager. */
+tq_status tq_prefix_cache_stats(tq_prefix_cache* pc, tq_prefix_stats* out);
+
+/* References held on one page (sequences + cache), -1 for a bad page id. */
+int32_t tq_prefix_cache_page_refs(tq_prefix_cache* pc, int32_t page);
 
 #ifdef __cplusplus
 }

@@ -22,7 +22,8 @@ CSRC = os.path.join(PKG, "csrc")
 OUT = os.path.join(PKG, "libtq.so")
 OBJ = os.path.join(ROOT, "_build", "libtq")
 
-SOURCES = ["append.cu", "decode.cu", "decode_tc.cu", "decode_noalloc.cu", "api.cu", "hbm.cu"]
+SOURCES = ["append.cu", "decode.cu", "decode_tc.cu", "decode_noalloc.cu", "api.cu", "hbm.cu",
+           "prefix_cache.cpp"]
 PER_FILE = {"append.cu": ["-fmad=false"]}
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
@@ -57,7 +58,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     os.makedirs(OBJ, exist_ok=True)
     objs = []
     for src in SOURCES:
-        obj = os.path.join(OBJ, src.replace(".cu", ".o"))
+        obj = os.path.join(OBJ, os.path.splitext(src)[0] + ".o")
         cmd = [nvcc(), *ARCH, *COMMON, *PER_FILE.get(src, []), "-c",
                os.path.join(CSRC, src), "-o", obj]
         if ptxas_info:

@@ -2,6 +2,7 @@
 // The contract of every entry point is stated in include/tq.h.
 #include <chrono>
 #include <cstdint>
+#include <new>
 #include <thread>
 
 #include <cuda_runtime.h>
@@ -41,6 +42,7 @@ int format_bits(int32_t f)
     case TQ_TURBO3: return 3;
     case TQ_TURBO4: return 4;
     case TQ_TURBO8: return 8;
+    case TQ_FP8: return 8;
     case TQ_BF16: return 16;
     default: return 0;
     }
@@ -173,6 +175,7 @@ TQ_API const char* tq_status_string(tq_status status)
     case TQ_ERR_TIMEOUT: return "TQ_ERR_TIMEOUT";
     case TQ_ERR_DEVICE_CHECK: return "TQ_ERR_DEVICE_CHECK";
     case TQ_ERR_WORKSPACE: return "TQ_ERR_WORKSPACE";
+    case TQ_ERR_NO_PAGES: return "TQ_ERR_NO_PAGES";
     default: return "TQ_ERR_UNKNOWN";
     }
 }
@@ -282,4 +285,71 @@ TQ_API tq_status tq_hbm_read(const void* src, size_t bytes, uint32_t* sink, void
     if (bytes == 0) return TQ_OK;
     if (!src || !sink || !aligned16(src) || (bytes & 15u)) return TQ_ERR_INVALID_ARG;
     return from_cuda(tq::launch_hbm_read(src, bytes, sink, static_cast<cudaStream_t>(stream)));
+}
+
+// ---------------------------------------------------------------- graphs
+struct tq_step_graph {
+    cudaGraph_t graph = nullptr;
+    cudaGraphExec_t exec = nullptr;
+};
+
+TQ_API tq_status tq_step_graph_create(const tq_cache* cache, const tq_step* step, void* stream,
+                                      tq_step_graph** graph)
+{
+    if (!graph || !step || !stream) return TQ_ERR_INVALID_ARG;    // not the legacy stream
+    *graph = nullptr;
+    const tq_status sc = check_cache(cache, cache ? cache->format != TQ_BF16 : true);
+    if (sc != TQ_OK) return sc;
+    const bool turbo = cache->format != TQ_BF16;
+    tq_status s = check_append(step->k, step->v, step->slot_mapping, step->num_tokens, cache, turbo);
+    if (s != TQ_OK) return s;
+    s = check_decode(step->q, cache, step->page_table, step->max_pages_per_seq, step->seq_lens,
+                     step->batch, step->q_len, step->num_q_heads, step->max_seq_len, step->out,
+                     step->workspace, step->workspace_bytes, turbo);
+    if (s != TQ_OK) return s;
+    tq_step_graph* g = new (std::nothrow) tq_step_graph();
+    if (!g) return TQ_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // relaxed capture: a kernel's first launch on a device also sets its
+    // shared-memory attribute, which this mode permits during capture
+    cudaError_t e = cudaStreamBeginCapture(st, cudaStreamCaptureModeRelaxed);
+    cudaError_t le = cudaSuccess;
+    if (e == cudaSuccess) {
+        const int64_t bb = block_bytes(cache->format, 128, cache->page_size);
+        if (step->num_tokens > 0)
+            le = turbo ? tq::launch_quantize_append(step->k, step->v, step->slot_mapping,
+                                                    step->num_tokens, cache->format, *cache, bb, st)
+                       : tq::launch_append_bf16(step->k, step->v, step->slot_mapping,
+                                                step->num_tokens, *cache, st);
+        if (le == cudaSuccess && step->batch > 0)
+            le = tq::launch_decode(step->q, *cache, bb, step->page_table, step->max_pages_per_seq,
+                                   step->seq_lens, step->batch, step->q_len, step->num_q_heads,
+                                   step->max_seq_len, step->out, step->workspace, st);
+        e = cudaStreamEndCapture(st, &g->graph);
+    }
+    if (e == cudaSuccess && le == cudaSuccess)
+        e = cudaGraphInstantiate(&g->exec, g->graph, 0);
+    if (e != cudaSuccess || le != cudaSuccess) {
+        if (g->exec) cudaGraphExecDestroy(g->exec);
+        if (g->graph) cudaGraphDestroy(g->graph);
+        delete g;
+        cudaGetLastError();                           // clear a launch error recorded in capture
+        return TQ_ERR_CUDA;
+    }
+    *graph = g;
+    return TQ_OK;
+}
+
+TQ_API tq_status tq_step_graph_launch(tq_step_graph* graph, void* stream)
+{
+    if (!graph || !graph->exec) return TQ_ERR_INVALID_ARG;
+    return from_cuda(cudaGraphLaunch(graph->exec, static_cast<cudaStream_t>(stream)));
+}
+
+TQ_API void tq_step_graph_destroy(tq_step_graph* graph)
+{
+    if (!graph) return;
+    if (graph->exec) cudaGraphExecDestroy(graph->exec);
+    if (graph->graph) cudaGraphDestroy(graph->graph);
+    delete graph;
 }

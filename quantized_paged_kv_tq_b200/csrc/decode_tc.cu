@@ -35,6 +35,7 @@
 // The epilogue merges the split (last CTA of a sequence/kv head wins an
 // atomic ticket and merges all splits), rotates back (H o / sqrt(d)) and
 // writes fp32 output.
+#include <algorithm>
 #include <cstdint>
 #include <math_constants.h>
 
@@ -79,14 +80,82 @@ struct TcArgs {
     int max_seq_len;
 };
 
-template <int BITS>
+template <int BITS, bool FP8 = false>
 struct TcFmt {
     static constexpr int CB = 16 * BITS;              // K row bytes (128 codes)
     static constexpr int L = (1 << (BITS - 1)) - 1;
     // codes come out of the unpacker in pairs (j, j + GB/2) of groups of GB
-    static constexpr int GB = BITS == 2 ? 16 : (BITS == 8 ? 4 : 8);
+    // (E4M3 codes convert in adjacent pairs: GB = 2)
+    static constexpr int GB = FP8 ? 2 : (BITS == 2 ? 16 : (BITS == 8 ? 4 : 8));
+    static constexpr float kDequant = FP8 ? 1.f / 448.f : 1.f / (float)L;   // code -> value / s
     static constexpr int kStage = 2 * kTile * (CB + 4);   // K and V blocks of one tile
 };
+
+// Two E4M3 codes (low byte first) -> f16x2 (exact: every E4M3 value is an f16)
+__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t two)
+{
+    uint32_t d;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"((unsigned short)(two & 0xFFFFu)));
+    return d;
+}
+
+// E4M3 K row (128 codes, chunks permuted as for 8-bit codes) -> tensor
+// memory columns [0, 64), codes in order: column j holds codes 2j, 2j + 1.
+__device__ __forceinline__ void k_row_to_tmem_fp8(const uint8_t* row, uint32_t taddr, int sw)
+{
+    uint32_t o[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint4 a = *reinterpret_cast<const uint4*>(row + 16 * ((2 * q) ^ sw));
+        const uint4 b = *reinterpret_cast<const uint4*>(row + 16 * ((2 * q + 1) ^ sw));
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            o[2 * i] = e4m3x2_f16x2(w[i]);
+            o[2 * i + 1] = e4m3x2_f16x2(w[i] >> 16);
+        }
+        tmem_st16(taddr + 16 * q, o);
+    }
+}
+
+// f16 NaN lanes -> 65504 (min.f16x2 returns the other operand of a NaN).
+// The encoder saturates, so a cached E4M3 code is never NaN; stage bytes past
+// the end of a sequence may be, and their zero weights must give zero products.
+__device__ __forceinline__ uint32_t finite_f16x2(uint32_t h)
+{
+    uint32_t d;
+    asm("min.f16x2 %0, %1, %2;" : "=r"(d) : "r"(h), "r"(0x7BFF7BFFu));
+    return d;
+}
+
+// E4M3 V codes of dimension `dim` for the tile's 128 tokens -> tensor memory
+// columns [0, 64) of this lane, tokens in order (vblk0, bb as v_col_to_tmem).
+__device__ __forceinline__ void v_col_to_tmem_fp8(const uint8_t* vblk0, int64_t bb, int lp,
+                                                  int dim, uint32_t taddr)
+{
+    const int P = 1 << lp;
+    uint32_t o[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int t0 = 32 * q, pg = t0 >> lp, in = t0 & (P - 1);
+        const uint8_t* row = vblk0 + pg * bb + (int64_t)dim * P;
+        uint4 x, y;
+        if (P >= 32) {
+            x = *reinterpret_cast<const uint4*>(row + in);
+            y = *reinterpret_cast<const uint4*>(row + in + 16);
+        } else {
+            x = *reinterpret_cast<const uint4*>(row);
+            y = *reinterpret_cast<const uint4*>(row + bb);
+        }
+        const uint32_t w[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            o[2 * i] = finite_f16x2(e4m3x2_f16x2(w[i]));
+            o[2 * i + 1] = finite_f16x2(e4m3x2_f16x2(w[i] >> 16));
+        }
+        tmem_st16(taddr + 16 * q, o);
+    }
+}
 
 // Index (dimension for K, token for V) held at K position k of an A operand,
 // i.e. the order the unpacker emits: pair c holds (perm(2c), perm(2c + 1)).
@@ -333,18 +402,18 @@ __device__ __forceinline__ void load_split_pids(int* s_pid, const TcArgs& a, int
 // un-normalised output rows [RG][128] (rotated domain); s_l: per-warp partial
 // row sums [4][16]; m_run: row maxima (log2 units).  A split that is the whole
 // sequence normalises, rotates back and writes; otherwise the partial goes to
-// the workspace and the last split CTA of the unit (atomic ticket) merges.
+// the workspace and the last split CTA of the unit (atomic ticket) merges;
+// `unit` indexes the (sequence, kv head, row group) in the workspace.
 // valid == false (the CTA gave up on a bounded wait; CTA-uniform): nothing
 // is read from sO, s_l or m_run; a split of a longer sequence still records
 // an empty partial (m = -inf) and takes its ticket, so the unit's counter
 // wraps back to zero and the workspace stays usable for later calls.
-template <int RG>
+template <int RG, bool ROT = true>
 __device__ __forceinline__ void tc_finish(const TcArgs& a, const float* sO, const float* s_l,
                                           const float* m_run, int* s_flag, int b, int kvh, int rg,
                                           int split, int nsplit, int nrows, int warp, int lane,
-                                          int tid, bool valid)
+                                          int tid, bool valid, int64_t unit)
 {
-    const int64_t unit = ((int64_t)b * gridDim.y + blockIdx.y);
     const int64_t part = unit * a.max_splits + split;
     const float rs = 0.08838834764831845f;
     if (!valid && nsplit == 1) return;
@@ -365,10 +434,11 @@ __device__ __forceinline__ void tc_finish(const TcArgs& a, const float* sO, cons
             const float inv = 1.f / Lsum;
 #pragma unroll
             for (int e = 0; e < 4; ++e) x[e] *= inv;
-            fwht128_lane(x, lane);
+            if (ROT) fwht128_lane(x, lane);
+            const float sc = ROT ? rs : 1.f;
             *reinterpret_cast<float4*>(a.out + (((int64_t)b * a.q_len + tq) * a.num_q_heads + h) *
                                                    kHeadDim + 4 * lane) =
-                make_float4(x[0] * rs, x[1] * rs, x[2] * rs, x[3] * rs);
+                make_float4(x[0] * sc, x[1] * sc, x[2] * sc, x[3] * sc);
         } else {
             *reinterpret_cast<float4*>(a.ws_o + (part * RG + rr) * kHeadDim + 4 * lane) =
                 make_float4(x[0], x[1], x[2], x[3]);
@@ -407,21 +477,24 @@ __device__ __forceinline__ void tc_finish(const TcArgs& a, const float* sO, cons
         }
         const float inv = 1.f / Lsum;
         float x[4] = {acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv};
-        fwht128_lane(x, lane);
+        if (ROT) fwht128_lane(x, lane);
+        const float sc = ROT ? rs : 1.f;
         const int R = rg * RG + rr;
         const int tq = R / a.group;
         const int h = kvh * a.group + (R - tq * a.group);
         *reinterpret_cast<float4*>(a.out + (((int64_t)b * a.q_len + tq) * a.num_q_heads + h) *
                                                kHeadDim + 4 * lane) =
-            make_float4(x[0] * rs, x[1] * rs, x[2] * rs, x[3] * rs);
+            make_float4(x[0] * sc, x[1] * sc, x[2] * sc, x[3] * sc);
     }
 }
 
-template <int BITS, int RG>
+// FP8: E4M3 codes (BITS = 8 layout), converted to f16; no rotation of the
+// query or of the output.
+template <int BITS, int RG, bool FP8 = false>
 __global__ void __launch_bounds__(kTcThreads, 4)
 k_decode_tc(const TcArgs a)
 {
-    using F = TcFmt<BITS>;
+    using F = TcFmt<BITS, FP8>;
     // RG query rows per CTA; operand columns: hi parts [0, RG), lo parts
     // [RG, 2 RG), zero padding up to NCOL (the MMA needs N >= 16)
     constexpr int NCOL = 2 * RG < 16 ? 16 : 2 * RG;
@@ -511,11 +584,12 @@ k_decode_tc(const TcArgs a)
             x[2] = bf16_bits_to_float(raw.y & 0xffffu);
             x[3] = bf16_bits_to_float(raw.y >> 16);
         }
-        fwht128_lane(x, lane);
+        if (!FP8) fwht128_lane(x, lane);
         float amax = 0.f;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            x[e] *= kLog2eTc / kHeadDim;       // (H q / sqrt d) . y / sqrt d = (H q) . y / d
+            // turbo: (H q / sqrt d) . y / sqrt d = (H q) . y / d; fp8: q . x / sqrt d
+            x[e] *= FP8 ? kLog2eTc * 0.08838834764831845f : kLog2eTc / kHeadDim;
             amax = fmaxf(amax, fabsf(x[e]));
         }
 #pragma unroll
@@ -572,7 +646,7 @@ k_decode_tc(const TcArgs a)
     int ev = 0;                                   // running V-scale exponent (biased)
     float vn = 1.f;                               // 2^(127 - ev)
     float vlimit = __uint_as_float(1u << 23);     // scales >= this raise ev
-    const float kinv = 1.f / (float)F::L;
+    const float kinv = F::kDequant;
     const int lim_min = seq_len - a.q_len + (rg * RG) / a.group;
     const int kpos = perm_inv<F::GB>(tid);        // this token's K position in PV
     bool aborted = false;
@@ -590,7 +664,8 @@ k_decode_tc(const TcArgs a)
         const int pg = tid >> a.lp, row = tid & (P - 1);
         const uint8_t* kblk = st + pg * 2 * a.block_bytes;     // stage: [page][K block, V block]
         const uint8_t* vblk = kblk + a.block_bytes;
-        k_row_to_tmem<BITS>(kblk + row * F::CB, t_lane, k_swizzle<BITS>(row));
+        if constexpr (FP8) k_row_to_tmem_fp8(kblk + row * F::CB, t_lane, k_swizzle<8>(row));
+        else k_row_to_tmem<BITS>(kblk + row * F::CB, t_lane, k_swizzle<BITS>(row));
         float ks = reinterpret_cast<const float*>(kblk + P * F::CB)[row] * kinv;
         float vs = reinterpret_cast<const float*>(vblk + P * F::CB)[row] * kinv;
         const int tok = tok0 + tid;
@@ -617,7 +692,8 @@ k_decode_tc(const TcArgs a)
         uint32_t sraw[NCOL];
 #pragma unroll
         for (int c = 0; c < NCOL; c += 16) tmem_ld16(t_lane + kColS + c, sraw + c);
-        v_col_to_tmem<BITS>(st + a.block_bytes, 2 * a.block_bytes, a.lp, tid, t_lane);
+        if constexpr (FP8) v_col_to_tmem_fp8(st + a.block_bytes, 2 * a.block_bytes, a.lp, tid, t_lane);
+        else v_col_to_tmem<BITS>(st + a.block_bytes, 2 * a.block_bytes, a.lp, tid, t_lane);
         tmem_wait_ld();
         const bool full_tile = tok0 + kTile - 1 <= lim_min;
         float sc[RG];
@@ -759,8 +835,8 @@ k_decode_tc(const TcArgs a)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
-    tc_finish<RG>(a, sO, s_l, m_run, s_flag, b, kvh, rg, split, nsplit, nrows, warp, lane, tid,
-                  ok);
+    tc_finish<RG, !FP8>(a, sO, s_l, m_run, s_flag, b, kvh, rg, split, nsplit, nrows, warp, lane,
+                        tid, ok, (int64_t)b * gridDim.y + blockIdx.y);
 }
 
 // ===================================================================
@@ -790,6 +866,7 @@ struct I8Fmt {
     static constexpr int F = BITS == 4 ? 16 : (BITS == 2 ? 64 : 1);
     static constexpr int kStage = 2 * kTile * (CB + 4);
 };
+
 
 // Shared-memory header of the integer kernel (bytes from the start).
 constexpr int kI8Pid = 1024;        // [128] split page ids
@@ -888,18 +965,20 @@ __device__ __forceinline__ void k_row_to_tmem_u8(const uint8_t* row, uint32_t ta
 // V codes of dimension `dim` for the tile's 128 tokens -> 32 words of
 // unsigned bytes in K-position order (registers; stored once the previous
 // PV product has drained).  vblk0 and bb as for v_col_to_tmem.
-template <int BITS>
-__device__ __forceinline__ void v_col_u8(const uint8_t* vblk0, int64_t bb, int lp, int dim,
-                                         uint32_t* o)
+template <int BITS, int Q0 = 0, int NQ = 4>
+__device__ __forceinline__ void v_col_u8(const uint8_t* vblk0, int bb, int lp, int dim,
+                                         uint32_t* o_all)
 {
     const int P = 1 << lp;
-    // 32 tokens per chunk: 16 bytes (4-bit), 8 bytes (2-bit), 32 bytes (8-bit)
+    // 32 tokens per chunk: 16 bytes (4-bit), 8 bytes (2-bit), 32 bytes (8-bit);
+    // chunks Q0 .. Q0 + NQ - 1 go to o_all[0 .. 8 NQ)
     const int row_bytes = P * BITS / 8;
+    uint32_t* o = o_all - 8 * Q0;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = Q0; q < Q0 + NQ; ++q) {
         const int t0 = 32 * q;
         const int pg = t0 >> lp, in = t0 & (P - 1);
-        const uint8_t* row = vblk0 + pg * bb + (int64_t)dim * row_bytes;
+        const uint8_t* row = vblk0 + pg * bb + dim * row_bytes;
         if constexpr (BITS == 4) {
             uint32_t w[4];
             if (P >= 32) {
@@ -1409,25 +1488,25 @@ k_decode_i8(const TcArgs a)
         tmem_dealloc(tmem, kTmemCols);
     }
     tc_finish<RG>(a, sO, s_l, m_run, s_flag, b, kvh, rg, split, nsplit, nrows, warp, lane, tid,
-                  ok);
+                  ok, (int64_t)b * gridDim.y + blockIdx.y);
 }
 
-template <int BITS, int RG>
+template <int BITS, int RG, bool FP8 = false>
 cudaError_t launch_tc(const TcArgs& a, dim3 grid, cudaStream_t stream)
 {
     constexpr int NCOL = 2 * RG < 16 ? 16 : 2 * RG;
-    const size_t smem = 1536 + 2 * 256 * NCOL + (size_t)kStages * TcFmt<BITS>::kStage;
+    const size_t smem = 1536 + 2 * 256 * NCOL + (size_t)kStages * TcFmt<BITS, FP8>::kStage;
     static int configured = 0;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 31 || !(configured & (1 << dev))) {
-        e = cudaFuncSetAttribute(k_decode_tc<BITS, RG>,
+        e = cudaFuncSetAttribute(k_decode_tc<BITS, RG, FP8>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         if (dev < 31) configured |= 1 << dev;
     }
-    k_decode_tc<BITS, RG><<<grid, kTcThreads, smem, stream>>>(a);
+    k_decode_tc<BITS, RG, FP8><<<grid, kTcThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
@@ -1511,6 +1590,10 @@ cudaError_t launch_decode_tc(const void* q, const tq_cache& c, int64_t block_byt
                            : launch_tc<3, 16>(a, grid, stream);
     case 4: TQ_I8(4);
     case 8: TQ_I8(8);
+    case TQ_FP8:
+        return rows == 4   ? launch_tc<8, 4, true>(a, grid, stream)
+               : rows == 8 ? launch_tc<8, 8, true>(a, grid, stream)
+                           : launch_tc<8, 16, true>(a, grid, stream);
     default: return cudaErrorInvalidValue;
     }
 #undef TQ_I8

@@ -30,6 +30,7 @@ TQ_ERR_CUDA = 3
 TQ_ERR_TIMEOUT = 4
 TQ_ERR_DEVICE_CHECK = 5
 TQ_ERR_WORKSPACE = 6
+TQ_ERR_NO_PAGES = 7
 
 TQ_TURBO2, TQ_TURBO3, TQ_TURBO4, TQ_TURBO8, TQ_BF16 = 2, 3, 4, 8, 16
 FORMATS = (TQ_TURBO2, TQ_TURBO3, TQ_TURBO4, TQ_TURBO8, TQ_BF16)
@@ -38,7 +39,11 @@ FORMATS = (TQ_TURBO2, TQ_TURBO3, TQ_TURBO4, TQ_TURBO8, TQ_BF16)
 SYMBOLS = ("tq_abi_version", "tq_status_string", "tq_page_block_bytes",
            "tq_quantize_append", "tq_append_bf16", "tq_decode_workspace_size",
            "tq_decode_workspace_init", "tq_paged_decode", "tq_paged_decode_bf16",
-           "tq_paged_decode_noalloc", "tq_read_device_error", "tq_hbm_copy", "tq_hbm_read")
+           "tq_paged_decode_noalloc", "tq_read_device_error", "tq_hbm_copy", "tq_hbm_read",
+           "tq_prefix_cache_create", "tq_prefix_cache_destroy", "tq_prefix_cache_begin",
+           "tq_prefix_cache_extend", "tq_prefix_cache_finish", "tq_prefix_cache_stats",
+           "tq_prefix_cache_page_refs", "tq_step_graph_create", "tq_step_graph_launch",
+           "tq_step_graph_destroy")
 
 
 class tq_cache(ctypes.Structure):
@@ -77,6 +82,48 @@ _lib.tq_hbm_copy.restype = _I
 _lib.tq_hbm_copy.argtypes = [_P, _P, _S, _P]
 _lib.tq_hbm_read.restype = _I
 _lib.tq_hbm_read.argtypes = [_P, _S, _P, _P]
+
+
+class tq_step(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("slot_mapping", ctypes.c_void_p), ("num_tokens", ctypes.c_int32),
+                ("q", ctypes.c_void_p), ("page_table", ctypes.c_void_p),
+                ("max_pages_per_seq", ctypes.c_int32), ("seq_lens", ctypes.c_void_p),
+                ("batch", ctypes.c_int32), ("q_len", ctypes.c_int32),
+                ("num_q_heads", ctypes.c_int32), ("max_seq_len", ctypes.c_int32),
+                ("out", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+
+_lib.tq_step_graph_create.restype = _I
+_lib.tq_step_graph_create.argtypes = [_CP, ctypes.POINTER(tq_step), _P, ctypes.POINTER(_P)]
+_lib.tq_step_graph_launch.restype = _I
+_lib.tq_step_graph_launch.argtypes = [_P, _P]
+_lib.tq_step_graph_destroy.restype = None
+_lib.tq_step_graph_destroy.argtypes = [_P]
+
+
+class tq_prefix_stats(ctypes.Structure):
+    _fields_ = [("free_pages", ctypes.c_int64), ("cached_blocks", ctypes.c_int64),
+                ("live_sequences", ctypes.c_int64), ("hit_tokens", ctypes.c_int64),
+                ("prompt_tokens", ctypes.c_int64), ("evictions", ctypes.c_int64)]
+
+
+_IP = ctypes.POINTER(ctypes.c_int32)
+_lib.tq_prefix_cache_create.restype = _P
+_lib.tq_prefix_cache_create.argtypes = [_I, _I, ctypes.c_int64]
+_lib.tq_prefix_cache_destroy.restype = None
+_lib.tq_prefix_cache_destroy.argtypes = [_P]
+_lib.tq_prefix_cache_begin.restype = _I
+_lib.tq_prefix_cache_begin.argtypes = [_P, _IP, _I, _IP, _I, _IP, _IP]
+_lib.tq_prefix_cache_extend.restype = _I
+_lib.tq_prefix_cache_extend.argtypes = [_P, _I, _I, _IP, _I]
+_lib.tq_prefix_cache_finish.restype = _I
+_lib.tq_prefix_cache_finish.argtypes = [_P, _I, _IP, _I]
+_lib.tq_prefix_cache_stats.restype = _I
+_lib.tq_prefix_cache_stats.argtypes = [_P, ctypes.POINTER(tq_prefix_stats)]
+_lib.tq_prefix_cache_page_refs.restype = _I
+_lib.tq_prefix_cache_page_refs.argtypes = [_P, _I]
 
 
 class TqError(RuntimeError):
@@ -260,3 +307,95 @@ def tq_hbm_copy(src: torch.Tensor, dst: torch.Tensor, stream=None) -> None:
 def tq_hbm_read(src: torch.Tensor, sink: torch.Tensor, stream=None) -> None:
     _check(_lib.tq_hbm_read(src.data_ptr(), src.numel() * src.element_size(), sink.data_ptr(),
                             _stream(stream)), "tq_hbm_read")
+
+
+class PrefixCache:
+    """Host-side prefix-block manager of a pool of `num_pages` pages
+    (tq_prefix_cache_* in include/tq.h).  Token ids are int32; page tables
+    come back as numpy int32 arrays for the caller to copy to the device."""
+
+    def __init__(self, num_pages: int, page_size: int = 16, max_cached_tokens: int = 0):
+        self.page_size = page_size
+        self.h = _lib.tq_prefix_cache_create(num_pages, page_size, max_cached_tokens)
+        if not self.h:
+            raise ValueError("tq_prefix_cache_create failed")
+
+    def __del__(self):
+        h = getattr(self, "h", None)
+        if h:
+            _lib.tq_prefix_cache_destroy(h)
+            self.h = None
+
+    @staticmethod
+    def _ids(tokens):
+        import numpy as np
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        return t, t.ctypes.data_as(_IP)
+
+    def begin(self, tokens, max_pages: int):
+        """(seq handle, cached token count, page table int32 [n pages])."""
+        import numpy as np
+        t, tp = self._ids(tokens)
+        pt = np.full(max_pages, -1, np.int32)
+        cached = ctypes.c_int32(0)
+        seq = ctypes.c_int32(-1)
+        _check(_lib.tq_prefix_cache_begin(self.h, tp, len(t), pt.ctypes.data_as(_IP), max_pages,
+                                          ctypes.byref(cached), ctypes.byref(seq)),
+               "tq_prefix_cache_begin")
+        n = -(-len(t) // self.page_size)
+        return seq.value, cached.value, pt[:n].copy()
+
+    def extend(self, seq: int, new_len: int, max_pages: int):
+        import numpy as np
+        pt = np.full(max_pages, -1, np.int32)
+        _check(_lib.tq_prefix_cache_extend(self.h, seq, new_len, pt.ctypes.data_as(_IP),
+                                           max_pages), "tq_prefix_cache_extend")
+        return pt[:-(-new_len // self.page_size)].copy()
+
+    def finish(self, seq: int, tokens) -> None:
+        t, tp = self._ids(tokens)
+        _check(_lib.tq_prefix_cache_finish(self.h, seq, tp, len(t)), "tq_prefix_cache_finish")
+
+    def stats(self) -> dict:
+        st = tq_prefix_stats()
+        _check(_lib.tq_prefix_cache_stats(self.h, ctypes.byref(st)), "tq_prefix_cache_stats")
+        return {name: getattr(st, name) for name, _ in tq_prefix_stats._fields_}
+
+    def page_refs(self, page: int) -> int:
+        return _lib.tq_prefix_cache_page_refs(self.h, page)
+
+
+class StepGraph:
+    """One append + decode step captured as a CUDA graph on `stream` (a
+    torch.cuda.Stream, not the default stream) with the given tensors fixed;
+    refresh the tensors' contents between launch() calls."""
+
+    def __init__(self, cache, stream, q, page_table, seq_lens, q_len, out, max_seq_len,
+                 k=None, v=None, slot_mapping=None, workspace=None):
+        B = q.shape[0]
+        if workspace is None and isinstance(cache, Cache):
+            workspace = cache.workspace(B, q_len, q.shape[2], max_seq_len)
+        T = k.shape[0] if k is not None else 0
+        self.step = tq_step(
+            k.data_ptr() if T else None, v.data_ptr() if T else None,
+            slot_mapping.data_ptr() if T else None, T,
+            _dev(q, torch.bfloat16, "q"), _dev(page_table, torch.int32, "page_table"),
+            page_table.shape[1], _dev(seq_lens, torch.int32, "seq_lens"), B, q_len, q.shape[2],
+            max_seq_len, _dev(out, torch.float32, "out"),
+            workspace.data_ptr() if workspace is not None else None,
+            workspace.numel() if workspace is not None else 0)
+        self._keep = (cache, q, page_table, seq_lens, out, k, v, slot_mapping, workspace)
+        h = ctypes.c_void_p()
+        _check(_lib.tq_step_graph_create(ctypes.byref(_desc(cache)), ctypes.byref(self.step),
+                                         _stream(stream), ctypes.byref(h)),
+               "tq_step_graph_create")
+        self.h = h.value
+
+    def launch(self, stream=None) -> None:
+        _check(_lib.tq_step_graph_launch(self.h, _stream(stream)), "tq_step_graph_launch")
+
+    def __del__(self):
+        h = getattr(self, "h", None)
+        if h:
+            _lib.tq_step_graph_destroy(h)
+            self.h = None

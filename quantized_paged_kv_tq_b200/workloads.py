@@ -183,6 +183,8 @@ def row_bytes(fmt: int, d: int = HEAD_DIM) -> int:
     """Cache bytes of one (token, kv head) row of K or of V: codes + scale."""
     if fmt == 16:
         return 2 * d
+    if fmt == 17:                       # fp8: one byte per code
+        return d + 4
     return d * fmt // 8 + 4
 
 

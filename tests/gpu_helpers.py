@@ -109,11 +109,19 @@ def check_close(got: np.ndarray, ref: np.ndarray, what: str = "") -> dict:
     return {"max_abs": max_abs, "rel_l2": rel_l2}
 
 
+FP8 = 17
+
+
+def code_bits(fmt: int) -> int:
+    """Bits per code of a cache format (fp8 codes are bytes)."""
+    return 8 if fmt == FP8 else fmt
+
+
 def k_unswizzle(rows: np.ndarray, off: int, fmt: int) -> np.ndarray:
     """Undo the documented 16-byte chunk permutation of a K token row at
     offset `off` in its page (include/tq.h: logical chunk c is stored at
     chunk c ^ w(off))."""
-    w = {2: (off >> 2) & 1, 4: (off >> 1) & 3, 8: off & 7}.get(fmt, 0)
+    w = {2: (off >> 2) & 1, 4: (off >> 1) & 3, 8: off & 7}.get(code_bits(fmt), 0)
     if w == 0:
         return rows
     n = rows.shape[-1] // 16
@@ -126,7 +134,7 @@ def k_pool_logical(kp: np.ndarray, fmt: int, P: int) -> np.ndarray:
     permutation undone (token rows in plain packed order, scales as they
     are)."""
     out = kp.copy()
-    cb = 128 * fmt // 8
+    cb = 128 * code_bits(fmt) // 8
     for r in range(P):
         out[..., r * cb:(r + 1) * cb] = k_unswizzle(kp[..., r * cb:(r + 1) * cb], r, fmt)
     return out

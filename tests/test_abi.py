@@ -33,8 +33,8 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_strings():
-    assert tq.abi_version() == 2
-    for s in range(7):
+    assert tq.abi_version() == 3
+    for s in range(8):
         assert tq.status_string(s).startswith("TQ_")
     assert tq.status_string(99) == "TQ_ERR_UNKNOWN"
 
@@ -183,8 +183,13 @@ def test_descriptor_layout_matches_the_c_header(tmp_path):
         "         offsetof(tq_cache, dev_error));\n"
         '  printf("%d %d %d %d %d %d\\n", TQ_TURBO2, TQ_TURBO3, TQ_TURBO4, TQ_TURBO8, TQ_BF16,\n'
         "         TQ_ABI_VERSION);\n"
-        '  printf("%d %d %d %d %d %d %d\\n", TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED,\n'
-        "         TQ_ERR_CUDA, TQ_ERR_TIMEOUT, TQ_ERR_DEVICE_CHECK, TQ_ERR_WORKSPACE);\n"
+        '  printf("%d %d %d %d %d %d %d %d\\n", TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED,\n'
+        "         TQ_ERR_CUDA, TQ_ERR_TIMEOUT, TQ_ERR_DEVICE_CHECK, TQ_ERR_WORKSPACE,\n"
+        "         TQ_ERR_NO_PAGES);\n"
+        '  printf("%zu %zu %zu %zu %zu %zu %zu\\n", sizeof(tq_prefix_stats),\n'
+        "         offsetof(tq_prefix_stats, free_pages), offsetof(tq_prefix_stats, cached_blocks),\n"
+        "         offsetof(tq_prefix_stats, live_sequences), offsetof(tq_prefix_stats, hit_tokens),\n"
+        "         offsetof(tq_prefix_stats, prompt_tokens), offsetof(tq_prefix_stats, evictions));\n"
         "  return 0;\n}\n")
     exe = tmp_path / "layout"
     subprocess.check_call([cc, "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o",
@@ -200,4 +205,24 @@ def test_descriptor_layout_matches_the_c_header(tmp_path):
                                                   tq.TQ_TURBO8, tq.TQ_BF16, tq.abi_version()]
     assert [int(x) for x in lines[2].split()] == [
         tq.TQ_OK, tq.TQ_ERR_INVALID_ARG, tq.TQ_ERR_UNSUPPORTED, tq.TQ_ERR_CUDA,
-        tq.TQ_ERR_TIMEOUT, tq.TQ_ERR_DEVICE_CHECK, tq.TQ_ERR_WORKSPACE]
+        tq.TQ_ERR_TIMEOUT, tq.TQ_ERR_DEVICE_CHECK, tq.TQ_ERR_WORKSPACE, tq.TQ_ERR_NO_PAGES]
+    S = tq.tq_prefix_stats
+    assert [int(x) for x in lines[3].split()] == [ctypes.sizeof(S)] + [
+        getattr(S, f).offset for f, _ in S._fields_]
+
+
+def test_step_graph_validation_on_the_host():
+    """The graph step checks its arguments like the two calls it captures
+    and refuses the legacy stream; nothing reaches the CUDA runtime."""
+    c = desc()
+    st = tq.tq_step()
+    h = ctypes.c_void_p()
+    create = tq.lib().tq_step_graph_create
+    assert create(ctypes.byref(c), ctypes.byref(st), None, ctypes.byref(h)) == tq.TQ_ERR_INVALID_ARG
+    st.batch, st.q_len, st.num_q_heads, st.max_seq_len = 1, 1, 8, 16
+    st.max_pages_per_seq = 1
+    # fake stream handle: validation fails (no q / out pointers) before any capture
+    assert create(ctypes.byref(c), ctypes.byref(st), FAKE, ctypes.byref(h)) == tq.TQ_ERR_INVALID_ARG
+    assert h.value is None
+    assert tq.lib().tq_step_graph_launch(None, None) == tq.TQ_ERR_INVALID_ARG
+    tq.lib().tq_step_graph_destroy(None)
