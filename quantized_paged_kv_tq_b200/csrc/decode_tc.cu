@@ -867,6 +867,11 @@ struct I8Fmt {
     static constexpr int kStage = 2 * kTile * (CB + 4);
 };
 
+// CTAs per SM of the integer kernel: tensor memory holds 4 (128 columns
+// each); with 4 query rows and 2- or 4-bit codes a fifth fits in registers
+// (96) and shared memory, stages its first tiles and query operand, and waits
+// in tcgen05.alloc until a running CTA frees its columns.
+constexpr int i8_ctas_per_sm(int bits, int rg) { return (rg <= 4 && bits != 8) ? 5 : 4; }
 
 // Shared-memory header of the integer kernel (bytes from the start).
 constexpr int kI8Pid = 1024;        // [128] split page ids
@@ -1045,7 +1050,7 @@ __device__ __forceinline__ float small_int_to_float(uint32_t v)
 }
 
 template <int BITS, int RG>
-__global__ void __launch_bounds__(kTcThreads, 4)
+__global__ void __launch_bounds__(kTcThreads, i8_ctas_per_sm(BITS, RG))
 k_decode_i8(const TcArgs a)
 {
     using F = I8Fmt<BITS>;
@@ -1104,15 +1109,7 @@ k_decode_i8(const TcArgs a)
         s_flag[0] = 0;
         fence_barrier_init();
     }
-    if (warp == 0) {
-        tmem_alloc(s_tmem, kTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
     __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *s_tmem;
-    const uint32_t t_lane = tmem + ((uint32_t)(32 * warp) << 16);
 
     // bulk copies of a tile, shared by the 4 warps
     auto issue_tile = [&](uint8_t* stg, uint64_t* bar, const int* pids, int t0) {
@@ -1199,7 +1196,17 @@ k_decode_i8(const TcArgs a)
 #pragma unroll
     for (int r = 0; r < RG; ++r) rowfac[r] = s_rowfac[r];
     fence_proxy_async_smem();
+    // tensor memory last: a CTA resident beyond the 4 whose columns fit
+    // waits here with its first tiles requested and its query operand staged
+    if (warp == 0) {
+        tmem_alloc(s_tmem, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    const uint32_t t_lane = tmem + ((uint32_t)(32 * warp) << 16);
     // accumulator start of S: registers for 4 rows, re-read from shared
     // memory for 8 (register pressure)
     constexpr int kInitRegs = RG <= 4 ? NS : 1;
@@ -1531,10 +1538,11 @@ cudaError_t launch_i8(const TcArgs& a, dim3 grid, cudaStream_t stream)
 
 }  // namespace
 
-// Query rows of one tensor-core CTA: 4, 8 or 16.  Up to 8 rows, 2-, 4- and
-// 8-bit codes go to the integer kernel; 3-bit codes, and every format with
-// more than 8 rows per kv head, to the f16 kernel (16 rows in one CTA, so
-// the kv head's pages are read once).
+// Query rows of one tensor-core CTA: 4, 8 or 16.  Up to 4 rows, 2-, 4- and
+// 8-bit codes go to the integer kernel; 3-bit and fp8 codes, and every format
+// with more than 4 rows per kv head, to the f16 kernel (its two columns per
+// row, against the integer kernel's four digit columns, make it the faster
+// one at 8 rows; 16 rows in one CTA read the kv head's pages once).
 int decode_tc_rows(int format, int G)
 {
     (void)format;
@@ -1580,7 +1588,7 @@ cudaError_t launch_decode_tc(const void* q, const tq_cache& c, int64_t block_byt
     const dim3 grid((unsigned)a.max_splits, (unsigned)(c.num_kv_heads * a.R), (unsigned)batch);
 #define TQ_I8(B)                                                                    \
     return rows == 4   ? launch_i8<B, 4>(a, grid, stream)                              \
-           : rows == 8 ? launch_i8<B, 8>(a, grid, stream)                              \
+           : rows == 8 ? launch_tc<B, 8>(a, grid, stream)                              \
                        : launch_tc<B, 16>(a, grid, stream)
     switch (c.format) {
     case 2: TQ_I8(2);
