@@ -281,7 +281,7 @@ def decode_kernel_label(fmt: int, G: int) -> str:
     rows = 4 if G <= 4 else (8 if G <= 8 else 16)
     if fmt == 17:
         return f"k_decode_tc<8,{rows},fp8>"
-    if fmt == 3 or rows == 16:
+    if fmt == 3 or rows > 4:
         return f"k_decode_tc<{fmt},{rows}>"
     return f"k_decode_i8<{fmt},{rows}>"
 

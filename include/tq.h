@@ -66,7 +66,11 @@
  * unspecified for the affected sequences.  No device code traps or asserts.
  *
  * Supported shapes: head_dim 128; page_size 16, 32 or 64; 1 <= q_len and
- * q_len * (num_q_heads / num_kv_heads) <= 64.
+ * q_len * (num_q_heads / num_kv_heads) <= 4096: one decode token, a verify
+ * window of draft tokens, or a chunk of prefill tokens (appended first, then
+ * attending causally over the cache).  Rows beyond 16 per kv head run as
+ * several 16-row groups (8 for a bf16 cache), each reading the kv head's
+ * pages.
  */
 #ifndef TQ_H
 #define TQ_H

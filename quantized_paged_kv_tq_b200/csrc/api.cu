@@ -31,7 +31,7 @@ cudaError_t launch_hbm_read(const void* src, size_t bytes, uint32_t* sink, cudaS
 
 namespace {
 
-constexpr int kMaxRows = 64;          // q_len * GQA group
+constexpr int kMaxRows = 4096;        // q_len * GQA group: a verify window or a prefill chunk
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

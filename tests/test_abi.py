@@ -102,7 +102,8 @@ def test_decode_validation():
     assert dec(c, q_len=0) == I
     assert dec(c, max_len=0) == I
     assert dec(c, maxp=255) == I                      # too few page-table columns
-    assert dec(c, q_len=17, Hq=32) == U               # 68 rows per kv head > 64
+    assert dec(c, q_len=1025, Hq=32) == U             # 4100 rows per kv head > 4096
+    assert dec(c, q_len=1024, Hq=32, max_len=1024, ws=None, ws_n=0) != U   # 4096 rows
     assert dec(c, B=70000) == U
     assert dec(c, q=FAKE + 4) == I
     assert dec(c, out=FAKE + 8) == I

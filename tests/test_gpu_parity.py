@@ -232,6 +232,24 @@ def test_causal_last_split_fully_masked_rows(q_len, lens):
     check_close(gpu_decode(w, 4, cache), oracle_decode(w, 4, np.arange(2)))
 
 
+@pytest.mark.parametrize("fmt,q_len,lens", [
+    (4, 64, (700, 2300)),        # 256 rows per kv head; the chunk crosses a split boundary
+    (3, 200, (2300, 200)),       # 800 rows; the second sequence is the chunk alone
+    (16, 96, (2200, 500)),       # bf16 cache: 8-row groups
+    (2, 256, (4096, 2400)),      # 1024 rows; a chunk at the end of two splits
+    (FP8, 48, (2100, 60)),
+])
+def test_chunked_prefill_over_quantised_pages(fmt, q_len, lens):
+    """A chunk of q_len prefill tokens, appended first, attends causally over
+    the cache: row t sees keys j <= seq_len - q_len + t.  Every row of every
+    chunk against the oracle."""
+    w = small(fmt, q_len=q_len, seq_lens=lens)
+    cache = gpu_fill(w, fmt)
+    check_close(gpu_decode(w, fmt, cache), oracle_decode(w, fmt, np.arange(len(lens))),
+                f"fmt {fmt} chunk {q_len}")
+    assert cache.read_error() == 0
+
+
 @pytest.mark.parametrize("fmt", (4, 2, 8))
 def test_mixed_lengths_in_one_batch(fmt):
     """Lengths of 1 token, exactly one split, one token past it, many
