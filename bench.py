@@ -646,6 +646,62 @@ def per_config(tq, dev, peak, resident_fill_inputs, appender, timed, bulk_append
     return rows
 
 
+def launch_only(args):
+    """Fill the workload's cache (bulk calls of up to 2^18 tokens), then
+    launch the decode, or the bulk append of the whole context in one call,
+    args.steps times with nothing else in between: the launch sequence an
+    ncu capture of one kernel selects from."""
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (libtq.so has no CPU path)")
+    from quantized_paged_kv_tq_b200 import build as tqbuild
+    tqbuild.build()
+    from quantized_paged_kv_tq_b200 import tq
+    dev = torch.device("cuda", 0)
+    w = W.make(args.workload)
+    fmt = args.fmt or w.formats[0]
+
+    def d_bf16(u16):
+        return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+
+    cache = tq.Cache(fmt, w.num_pages, w.num_kv_heads, w.page_size, device=dev)
+
+    def fill(k, v, s):
+        if fmt == 16:
+            tq.tq_append_bf16(k, v, s, cache)
+        else:
+            tq.tq_quantize_append(k, v, s, fmt, cache)
+
+    if args.launch_only == "append":
+        parts = list(w.iter_fill(1 << 18))
+        s_d = torch.cat([torch.from_numpy(s.astype(np.int64)) for s, _, _ in parts]).to(dev)
+        k_d = torch.cat([d_bf16(k) for _, k, _ in parts])
+        v_d = torch.cat([d_bf16(v) for _, _, v in parts])
+        del parts
+        for _ in range(args.steps):
+            fill(k_d, v_d, s_d)
+    else:
+        for s, k, v in w.iter_fill(1 << 18):
+            fill(d_bf16(k), d_bf16(v), torch.from_numpy(s.astype(np.int64)).to(dev))
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        q = d_bf16(w.queries())
+        pt = torch.from_numpy(w.page_table).to(dev)
+        sl = torch.from_numpy(w.seq_lens).to(dev)
+        out = torch.empty((w.batch, w.q_len, w.num_q_heads, w.head_dim), dtype=torch.float32,
+                          device=dev)
+        ws = cache.workspace(w.batch, w.q_len, w.num_q_heads, w.max_seq_len)
+        decode = tq.tq_paged_decode_bf16 if fmt == 16 else tq.tq_paged_decode
+        for _ in range(args.steps):
+            decode(q, cache, pt, sl, w.q_len, out, max_seq_len=w.max_seq_len, workspace=ws)
+    torch.cuda.synchronize()
+    err = cache.read_error()
+    print(f"launch-only {args.launch_only} {args.workload} format {fmt}: {args.steps} launches, "
+          f"device error word {err:#x}")
+    return 0 if err == 0 else 1
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -657,7 +713,13 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip the per-configuration decode and bulk-append timings")
+    ap.add_argument("--launch-only", choices=("decode", "append"),
+                    help="for a profiler: fill the workload's cache, then launch only the "
+                         "decode (or the bulk quantise-append of the whole context) --steps "
+                         "times, untimed, and print one status line")
     args = ap.parse_args(argv)
+    if args.launch_only:
+        return launch_only(args)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

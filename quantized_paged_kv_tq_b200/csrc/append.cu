@@ -151,18 +151,25 @@ __device__ __forceinline__ void quantize32(const float y[32], float s, uint32_t 
     }
     bool slow = !(s > 2.350988701644575e-38f * 0.5f && s < 4.2535295865117308e37f);  // 2^-126 .. 2^125
     const float r = __frcp_rn(s);
+    // |q| < 2^22: q + 1.5 2^23 lies in [2^23, 2^24), where the fp32 spacing is
+    // 1, so the sum is rounded to the nearest integer n (ties to even, as
+    // rintf), its bit pattern is that of 1.5 2^23 plus n, and subtracting
+    // 1.5 2^23 again gives n exactly
+    constexpr float kRound = 12582912.f;                 // 1.5 2^23 = 0x4B400000
+    constexpr uint32_t kBias = 0x4B400000u - (uint32_t)L; // bits(kRound + n) - kBias = n + L
     const unsigned long long L2 = pk2((float)L, (float)L), r2 = pk2(r, r);
+    const unsigned long long m2 = pk2(kRound, kRound);
 #pragma unroll
     for (int i = 0; i < 32; i += 2) {
         const unsigned long long t2 = mul2(pk2(y[i], y[i + 1]), L2);
-        float q0, q1;
-        up2(mul2(t2, r2), q0, q1);
-        const float r0 = rintf(q0), r1 = rintf(q1);
-        float d0, d1;
-        up2(sub2(pk2(q0, q1), pk2(r0, r1)), d0, d1);
+        const unsigned long long q2 = mul2(t2, r2);
+        const unsigned long long n2 = add2(q2, m2);          // kRound + rint(q)
+        float d0, d1, n0, n1;
+        up2(sub2(q2, sub2(n2, m2)), d0, d1);                  // q - rint(q), exact
         slow |= !(fabsf(d0) <= 0.49993896484375f) | !(fabsf(d1) <= 0.49993896484375f);  // 0.5 - 2^-14
-        u[i] = (uint32_t)((int)r0 + L);
-        u[i + 1] = (uint32_t)((int)r1 + L);
+        up2(n2, n0, n1);
+        u[i] = __float_as_uint(n0) - kBias;
+        u[i + 1] = __float_as_uint(n1) - kBias;
     }
     if (slow) {
 #pragma unroll
