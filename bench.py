@@ -112,9 +112,9 @@ def decode_sources_sha256() -> str:
 
 
 def profiled_traffic(kernel: str):
-    """dram read+write bytes per launch recorded in profiles/<kernel>*.txt,
-    valid only while the decode sources are unchanged (their sha256 is
-    recorded as decode_src_sha256)."""
+    """dram read+write bytes per launch recorded in profiles/<kernel>*.md
+    (e.g. k_decode_i8_target64x8k_turbo4.md), valid only while the decode
+    sources are unchanged (their sha256 is recorded as decode_src_sha256)."""
     sha = decode_sources_sha256()
     pdir = os.path.join(ROOT, "profiles")
     if not os.path.isdir(pdir):
@@ -563,7 +563,10 @@ def run_ours(args):
                         "decode_vs_inrun_read": achieved / read_gbs,
                         "append_bulk": main_bulk["frac_of_hbm"]},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": profiled_traffic("decode"),
+                     "frac": achieved / peak,
+                     "traffic": profiled_traffic(
+                         f"{decode_kernel_label(fmt, w.q_len * w.group).split('<')[0]}_"
+                         f"{args.workload}_{FORMAT_NAMES[fmt]}"),
                      "peak_source": f"hbm_gbs of {peak_kind}",
                      "algorithmic_bytes_per_launch": kv_bytes},
         "e2e": {"value": world * kv_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
@@ -576,6 +579,7 @@ def run_ours(args):
     if not args.no_per_config:
         line["per_config"] = per_config(tq, dev, peak, resident_fill_inputs, appender, timed,
                                         bulk_append_report)
+        line["extra"] = extra_rows(tq, dev, peak, timed)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, fmt)
     if world > 1:
@@ -643,6 +647,102 @@ def per_config(tq, dev, peak, resident_fill_inputs, appender, timed, bulk_append
             torch.cuda.empty_cache()
         del s_d, k_d, v_d, q, pt, sl, out
         torch.cuda.empty_cache()
+    return rows
+
+
+def extra_rows(tq, dev, peak, timed):
+    """Two measurements beside the per-configuration decodes: a chunk of
+    prefill tokens attending causally over a quantised context (q_len 256,
+    1024 rows per kv head), and the append + decode step of batch8 eager
+    against replayed as one CUDA graph.  L2 flushed before every launch."""
+    import torch
+    rows = []
+
+    def d_bf16(u16):
+        return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+
+    # ---- prefill chunk
+    w = W.custom(batch=4, num_q_heads=32, num_kv_heads=8, page_size=16, q_len=256,
+                 seq_lens=(4096,) * 4, fmt=4, seed=9)
+    cache = tq.Cache(4, w.num_pages, w.num_kv_heads, w.page_size, device=dev)
+    for slots, k, v in w.iter_fill(1 << 16):
+        tq.tq_quantize_append(d_bf16(k), d_bf16(v), torch.from_numpy(slots.astype(np.int64)).to(dev),
+                              4, cache)
+    q = d_bf16(w.queries())
+    pt = torch.from_numpy(w.page_table).to(dev)
+    sl = torch.from_numpy(w.seq_lens).to(dev)
+    out = torch.empty((w.batch, w.q_len, w.num_q_heads, w.head_dim), dtype=torch.float32,
+                      device=dev)
+    ws = cache.workspace(w.batch, w.q_len, w.num_q_heads, w.max_seq_len)
+
+    def dec():
+        tq.tq_paged_decode(q, cache, pt, sl, w.q_len, out, max_seq_len=w.max_seq_len, workspace=ws)
+
+    for _ in range(3):
+        dec()
+    ms, ms_min = timed(dec, 20, flush=True)
+    if cache.read_error():
+        raise SystemExit("prefill chunk: device error word set")
+    G = w.q_len * w.group
+    # (row, visible key) pairs: row t of the chunk sees seq_len - q_len + t + 1 keys
+    pairs = sum(w.group * (int(L) - w.q_len + t + 1) for L in w.seq_lens for t in range(w.q_len))
+    pairs *= w.num_kv_heads
+    flops = pairs * 4 * w.head_dim                      # QK and PV, 2 flops per MAC
+    uniq = int(w.seq_lens.sum()) * w.num_kv_heads * 2 * W.row_bytes(4)
+    rows.append({"workload": "prefill chunk: batch 4 x 4096-token context, the last 256 tokens "
+                             "a prefill chunk, 32 q / 8 kv heads, page 16, turbo4",
+                 "kernel": decode_kernel_label(4, G), "rows_per_kv_head": G,
+                 "decode_us": ms * 1e3, "decode_us_min": ms_min * 1e3,
+                 "chunk_tokens_per_s": w.batch * w.q_len / (ms * 1e-3),
+                 "tflops": flops / (ms * 1e-3) / 1e12, "flops": flops,
+                 "unique_kv_bytes": uniq, "unique_frac_of_hbm": uniq / (ms * 1e-3) / 1e9 / peak,
+                 "l2": "flushed before every timed launch; the 16-row groups re-read a kv "
+                       "head's pages, mostly from L2"})
+    del cache, ws, q, out
+    torch.cuda.empty_cache()
+
+    # ---- batch8 step: eager against one CUDA graph
+    w = W.make("batch8")
+    cache = tq.Cache(4, w.num_pages, w.num_kv_heads, w.page_size, device=dev)
+    for slots, k, v in w.iter_fill(1 << 16, upto=w.seq_lens - 1):
+        tq.tq_quantize_append(d_bf16(k), d_bf16(v), torch.from_numpy(slots.astype(np.int64)).to(dev),
+                              4, cache)
+    new_slots = torch.from_numpy(np.array([w.slots_of(b, [int(w.seq_lens[b]) - 1])[0]
+                                           for b in range(w.batch)], np.int64)).to(dev)
+    k, v = w.new_tokens(0, w.batch)
+    nk, nv = d_bf16(k), d_bf16(v)
+    q = d_bf16(w.queries())
+    pt = torch.from_numpy(w.page_table).to(dev)
+    sl = torch.from_numpy(w.seq_lens).to(dev)
+    out = torch.empty((w.batch, w.q_len, w.num_q_heads, w.head_dim), dtype=torch.float32,
+                      device=dev)
+    ws = cache.workspace(w.batch, w.q_len, w.num_q_heads, w.max_seq_len)
+    side = torch.cuda.Stream(device=dev)
+    g = tq.StepGraph(cache, side, q, pt, sl, w.q_len, out, w.max_seq_len, k=nk, v=nv,
+                     slot_mapping=new_slots, workspace=ws)
+
+    def eager():
+        tq.tq_quantize_append(nk, nv, new_slots, 4, cache)
+        tq.tq_paged_decode(q, cache, pt, sl, w.q_len, out, max_seq_len=w.max_seq_len,
+                           workspace=ws)
+
+    def graph():
+        g.launch(torch.cuda.current_stream())
+
+    for _ in range(3):
+        eager()
+        graph()
+    ms_e, _ = timed(eager, 50, flush=True)
+    ms_g, _ = timed(graph, 50, flush=True)
+    if cache.read_error():
+        raise SystemExit("graph step: device error word set")
+    rows.append({"workload": "batch8 step: append 1 token per sequence + decode, 8 x 4096, "
+                             "32 q / 8 kv heads, page 16, turbo4",
+                 "eager_us": ms_e * 1e3, "graph_us": ms_g * 1e3,
+                 "l2": "flushed before every timed step"})
+    del g, cache, ws
+    torch.cuda.empty_cache()
     return rows
 
 

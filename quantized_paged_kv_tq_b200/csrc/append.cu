@@ -40,7 +40,9 @@ constexpr int kQaThreads = 256;
 constexpr int kQaWin = 64;             // tokens per window before alignment (large calls)
 constexpr int kQaMaxWin = 128;         // staging capacity: kQaWin + page_size - 1 <= 127
 constexpr int kQaPass = 32;            // tokens per pass (x K and V = 64 vectors)
-constexpr int kVRow = 160;             // staging row: window tokens, XOR 8 (dim / 32), + one group
+// staging row: window tokens, XOR 8 (dim / 32), + one group (>= 160); 168 so
+// that the V writer's 8-byte reads of rows 2 apart spread over the banks
+constexpr int kVRow = 168;
 constexpr int kQaStages = 3;           // input ring: each thread's next passes, by cp.async
 constexpr int kQaInBytes = kQaStages * kQaThreads * 64;
 
@@ -233,7 +235,7 @@ k_quantize_append(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v
                   uint8_t* __restrict__ pool, uint32_t* err)
 {
     constexpr int CB = kHeadDim * BITS / 8;            // K row bytes
-    extern __shared__ __align__(16) uint8_t s_in[];    // [stage][thread][64 B] input ring
+    extern __shared__ __align__(16) uint8_t s_in[];    // [stage][chunk][thread][16 B] input ring
     __shared__ __align__(16) uint8_t s_v[kHeadDim * kVRow];   // [dim][token ^ 8 (dim / 32)]
     __shared__ int s_page[kQaMaxWin], s_off[kQaMaxWin], s_run[kQaMaxWin];
     __shared__ int s_rs[kQaMaxWin], s_rlen[kQaMaxWin];  // runs: first window token, length
@@ -462,9 +464,10 @@ k_quantize_append(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v
             if (tk < n) {
                 const uint16_t* src = (which ? v : k) +
                                       ((w0 + tk) * num_kv_heads + head0 + hh) * kHeadDim + 32 * q;
-                uint8_t* dst = s_in + ((pidx % kQaStages) * kQaThreads + tid) * 64;
+                // ring slot [stage][chunk][thread]: a warp's 16-byte chunks are contiguous
+                uint8_t* dst = s_in + ((pidx % kQaStages) * 4 * kQaThreads + tid) * 16;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) cp_async16(dst + 16 * c, src + 8 * c);
+                for (int c = 0; c < 4; ++c) cp_async16(dst + c * kQaThreads * 16, src + 8 * c);
             }
         }
         cp_async_commit();
@@ -480,11 +483,11 @@ k_quantize_append(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v
         const bool live = tk < n && s_page[tk] >= 0;
         float x[32];
         if (tk < n) {
-            const uint4* src = reinterpret_cast<const uint4*>(
-                s_in + ((pidx % kQaStages) * kQaThreads + tid) * 64);
+            const uint4* src = reinterpret_cast<const uint4*>(s_in) +
+                               (pidx % kQaStages) * 4 * kQaThreads + tid;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const uint4 raw = src[c];
+                const uint4 raw = src[c * kQaThreads];
                 const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
