@@ -278,6 +278,8 @@ def decode_kernel_label(fmt: int, G: int) -> str:
     format and G = q_len x GQA rows per kv head (a label for the report)."""
     if fmt == 16:
         return "k_decode<16>"
+    if fmt != 17 and G >= 128:
+        return f"k_prefill_tc<{fmt}>"
     rows = 4 if G <= 4 else (8 if G <= 8 else 16)
     if fmt == 17:
         return f"k_decode_tc<8,{rows},fp8>"

@@ -68,9 +68,11 @@
  * Supported shapes: head_dim 128; page_size 16, 32 or 64; 1 <= q_len and
  * q_len * (num_q_heads / num_kv_heads) <= 4096: one decode token, a verify
  * window of draft tokens, or a chunk of prefill tokens (appended first, then
- * attending causally over the cache).  Rows beyond 16 per kv head run as
- * several 16-row groups (8 for a bf16 cache), each reading the kv head's
- * pages.
+ * attending causally over the cache).  With a turbo format, 128 or more
+ * rows per kv head run on a query-major kernel (128 rows per CTA, each K/V
+ * tile dequantised once per 128 rows, no split workspace); fewer rows beyond
+ * 16 run as several 16-row groups (8 for a bf16 cache, 16 for fp8), each
+ * reading the kv head's pages.
  */
 #ifndef TQ_H
 #define TQ_H

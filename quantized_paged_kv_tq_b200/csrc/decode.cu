@@ -677,9 +677,12 @@ int decode_row_groups(int format, int G)
 }
 
 // Workspace: [counters (256-byte aligned)][m,l partials][O partials]
+bool decode_uses_prefill(int format, int G);
+
 size_t decode_workspace_bytes(int batch, int num_kv_heads, int G, int max_seq_len, int page_size,
                               int format)
 {
+    if (decode_uses_prefill(format, G)) return 0;       // rows written directly
     const int st = decode_split_tokens(page_size);
     const int64_t max_splits = (max_seq_len + st - 1) / st;
     if (max_splits <= 1) return 0;

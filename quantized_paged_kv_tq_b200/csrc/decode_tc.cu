@@ -219,9 +219,10 @@ __device__ __forceinline__ void pairs3(uint32_t g, uint32_t* o)
 }
 
 // K row of one token (128 codes; 16-byte chunks permuted by `sw`, see
-// k_swizzle) -> tensor memory columns [col, col + 64).
-template <int BITS>
-__device__ __forceinline__ void k_row_to_tmem(const uint8_t* row, uint32_t taddr, int sw)
+// k_swizzle) as 64 words of f16 pairs, handed to sink(c, o) 16 words at a
+// time (words c .. c + 15).
+template <int BITS, class Sink>
+__device__ __forceinline__ void k_row_unpack(const uint8_t* row, int sw, Sink&& sink)
 {
     uint32_t o[16];
     auto chunk = [&](int c) { return *reinterpret_cast<const uint4*>(row + 16 * (c ^ sw)); };
@@ -233,7 +234,7 @@ __device__ __forceinline__ void k_row_to_tmem(const uint8_t* row, uint32_t taddr
             pairs4(w.y, o + 4);
             pairs4(w.z, o + 8);
             pairs4(w.w, o + 12);
-            tmem_st16(taddr + 16 * q, o);
+            sink(16 * q, o);
         }
     } else if constexpr (BITS == 8) {
 #pragma unroll
@@ -242,7 +243,7 @@ __device__ __forceinline__ void k_row_to_tmem(const uint8_t* row, uint32_t taddr
             const uint4 b = chunk(2 * q + 1);
             pairs8(a.x, o); pairs8(a.y, o + 2); pairs8(a.z, o + 4); pairs8(a.w, o + 6);
             pairs8(b.x, o + 8); pairs8(b.y, o + 10); pairs8(b.z, o + 12); pairs8(b.w, o + 14);
-            tmem_st16(taddr + 16 * q, o);
+            sink(16 * q, o);
         }
     } else if constexpr (BITS == 2) {
 #pragma unroll
@@ -250,10 +251,10 @@ __device__ __forceinline__ void k_row_to_tmem(const uint8_t* row, uint32_t taddr
             const uint4 w = chunk(q);
             pairs2(w.x, o);
             pairs2(w.y, o + 8);
-            tmem_st16(taddr + 32 * q, o);
+            sink(32 * q, o);
             pairs2(w.z, o);
             pairs2(w.w, o + 8);
-            tmem_st16(taddr + 32 * q + 16, o);
+            sink(32 * q + 16, o);
         }
     } else {  // 3 bits: 48-byte row, 12 words, 16 groups of 8 codes
 #pragma unroll
@@ -265,17 +266,25 @@ __device__ __forceinline__ void k_row_to_tmem(const uint8_t* row, uint32_t taddr
             pairs3(prmt(W0, W1, 0x6543u), o + 4);
             pairs3(prmt(W1, W2, 0x5432u), o + 8);
             pairs3(W2 >> 8, o + 12);
-            tmem_st16(taddr + 16 * q, o);
+            sink(16 * q, o);
         }
     }
 }
 
-// V codes of dimension `dim` for the 128 tokens of a tile -> tensor memory
-// columns [0, 64) of this thread's lane.  vblk0: V block of the tile's first
-// page in the stage; the V blocks of later pages follow every `bb` bytes.
+// ... into tensor memory columns [0, 64) of this thread's lane
 template <int BITS>
-__device__ __forceinline__ void v_col_to_tmem(const uint8_t* vblk0, int64_t bb, int lp, int dim,
-                                              uint32_t taddr)
+__device__ __forceinline__ void k_row_to_tmem(const uint8_t* row, uint32_t taddr, int sw)
+{
+    k_row_unpack<BITS>(row, sw, [&](int c, const uint32_t* o) { tmem_st16(taddr + c, o); });
+}
+
+// V codes of dimension `dim` for the 128 tokens of a tile as 64 words of
+// f16 pairs, handed to sink(c, o) 16 words at a time.  vblk0: V block of the
+// tile's first page in the stage; the V blocks of later pages follow every
+// `bb` bytes.
+template <int BITS, class Sink>
+__device__ __forceinline__ void v_col_unpack(const uint8_t* vblk0, int64_t bb, int lp, int dim,
+                                             Sink&& sink)
 {
     const int P = 1 << lp;
     uint32_t o[16];
@@ -339,8 +348,17 @@ __device__ __forceinline__ void v_col_to_tmem(const uint8_t* vblk0, int64_t bb, 
                 pairs3((uint32_t)(v64 >> 24) & 0xFFFFFFu, o + 8 * h + 4);
             }
         }
-        tmem_st16(taddr + 16 * q, o);
+        sink(16 * q, o);
     }
+}
+
+// ... into tensor memory columns [0, 64) of this thread's lane
+template <int BITS>
+__device__ __forceinline__ void v_col_to_tmem(const uint8_t* vblk0, int64_t bb, int lp, int dim,
+                                              uint32_t taddr)
+{
+    v_col_unpack<BITS>(vblk0, bb, lp, dim,
+                       [&](int c, const uint32_t* o) { tmem_st16(taddr + c, o); });
 }
 
 // Bulk copies of one tile's pages into a stage (warp 0): one copy per page of
@@ -1536,6 +1554,389 @@ cudaError_t launch_i8(const TcArgs& a, dim3 grid, cudaStream_t stream)
     return cudaGetLastError();
 }
 
+// ===================================================================
+// Query-major kernel for long verify windows and prefill chunks (turbo
+// formats, G = q_len x GQA >= 128 rows per kv head).
+//
+// One CTA (128 threads) owns 128 query rows of one (sequence, kv head) and
+// walks every key tile its rows may see (causal), so each K/V tile is
+// dequantised once for 128 rows instead of once per 16-row group:
+//   1. token t unpacks its K row, and dimension t its V column, into exact
+//      f16 integers in shared memory, in the canonical K-major layout (8x8
+//      core matrices) of the MMA's B operand; the tile's K and V scales go
+//      to shared memory too.
+//   2. one thread issues S[128 rows][128 keys] = Q' K^T: A = Q' in tensor
+//      memory (the rotated query, prescaled per row, split into f16 hi and
+//      lo parts: two MMA chains into one fp32 accumulator).
+//   3. thread r owns row r: it reads its scores (twice: the row maximum,
+//      then the weights), scales them by s_k / L and the row factor, masks
+//      keys beyond its causal limit, and runs an online softmax with a lazy
+//      maximum (a warp rescales its rows of O only when one of them gains
+//      more than 2^8).  P' = p s_v / L 2^(127 - ev), split hi/lo in f16, goes
+//      to tensor memory as the A operand of the PV product (keys in the V
+//      unpacker's pair order).
+//   4. one thread issues O[128 rows][128 dims] += P' V (two chains).
+// The epilogue normalises each row, rotates it back (a 128-point FWHT in
+// the thread's registers) and writes it; there is no split merge.
+// Tensor memory: Q' hi/lo 128 columns, S 128, O 128, P' hi/lo 128.
+// ===================================================================
+constexpr int kPfRows = 128;
+constexpr uint32_t kPfColQ = 0, kPfColS = 128, kPfColO = 256, kPfColP = 384;
+constexpr uint32_t kPfTmemCols = 512;
+// shared memory (bytes from the start)
+constexpr int kPfKs = 128;          // [128] K scales of the tile, / L
+constexpr int kPfVs = 640;          // [128] V scales of the tile, / L
+constexpr int kPfKdeq = 2048;       // [128 keys x 128 dims] f16, B of S
+constexpr int kPfVdeq = kPfKdeq + 32768;   // [128 dims x 128 keys] f16, B of O
+constexpr int kPfRing = kPfVdeq + 32768;   // [kStages] tile stages
+
+// K-major core-matrix offset (bytes) of element (n, k) of a [128 x 128] f16
+// B operand: 8x8 core matrices of 128 bytes, N-adjacent ones 128 bytes
+// apart, K-adjacent ones 16 x 128 bytes apart.
+__device__ __forceinline__ int pf_b_offset(int n, int k)
+{
+    return ((k >> 3) * 16 + (n >> 3)) * 128 + (n & 7) * 16 + (k & 7) * 2;
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(kTcThreads, 1)
+k_prefill_tc(const TcArgs a)
+{
+    using F = TcFmt<BITS>;
+    // f32 accumulate, f16 A (tensor memory) and B (shared, K-major), M = 128, N = 128
+    constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(128 >> 3) << 17) | (8u << 24);
+    constexpr uint32_t kLbo = 16 * 128;             // K-adjacent core matrices
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);              // [kStages]
+    uint64_t* bar_s = full + kStages;
+    uint64_t* bar_o = bar_s + 1;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + 64);
+    int* s_flag = reinterpret_cast<int*>(smem + 68);
+    float* s_ks = reinterpret_cast<float*>(smem + kPfKs);
+    float* s_vs = reinterpret_cast<float*>(smem + kPfVs);
+    uint8_t* kdeq = smem + kPfKdeq;
+    uint8_t* vdeq = smem + kPfVdeq;
+    uint8_t* ring = smem + kPfRing;
+
+    const int rb = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int seq_len = a.seq_lens[b];
+    if (seq_len < a.q_len || seq_len > a.max_seq_len) {
+        if (rb == 0 && kvh == 0 && tid == 0) report_error(a.err, TQ_ERR_DEVICE_CHECK, kErrSeqLen);
+        return;
+    }
+    const int P = a.page_size;
+    // this thread's row, its causal limit; the block's last visible key
+    const int R = rb * kPfRows + tid;
+    const bool row_ok = R < a.G;
+    const int tq = row_ok ? R / a.group : 0;
+    const int h = kvh * a.group + (R - tq * a.group);
+    const int lim = row_ok ? seq_len - a.q_len + tq : -1;
+    const int r_last = min(a.G, (rb + 1) * kPfRows) - 1;
+    const int nkeys = seq_len - a.q_len + r_last / a.group + 1;     // <= seq_len
+    const int ntiles = (nkeys + kTile - 1) / kTile;
+    const int32_t* pt = a.page_table + (int64_t)b * a.max_pages;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+        mbar_init(bar_s, 1);
+        mbar_init(bar_o, 1);
+        s_flag[0] = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(s_tmem, kPfTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    const uint32_t t_lane = tmem + ((uint32_t)(32 * warp) << 16);
+
+    if (warp == 0)
+        for (int s = 0; s < kStages && s < ntiles; ++s)
+            issue_tile_tc(ring + s * F::kStage, &full[s], a, pt + ((s * kTile) >> a.lp), kvh,
+                          min(kTile, nkeys - s * kTile), lane);
+
+    // ---- Q' of this row: rotate (128-point FWHT in registers), log2 scale,
+    // power-of-two prescale, f16 hi + lo in the K unpacker's dimension order
+    float rowfac = 1.f;
+    {
+        float x[kHeadDim];
+        if (row_ok) {
+            const uint4* src = reinterpret_cast<const uint4*>(
+                a.q + (((int64_t)b * a.q_len + tq) * a.num_q_heads + h) * kHeadDim);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const uint4 w = __ldg(src + c);
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    x[8 * c + 2 * e] = bf16_bits_to_float(ww[e] & 0xffffu);
+                    x[8 * c + 2 * e + 1] = bf16_bits_to_float(ww[e] >> 16);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < kHeadDim; ++i) x[i] = 0.f;
+        }
+#pragma unroll
+        for (int hs = 1; hs < kHeadDim; hs <<= 1)
+#pragma unroll
+            for (int i = 0; i < kHeadDim; ++i)
+                if (!(i & hs)) {
+                    const float u = x[i], v = x[i + hs];
+                    x[i] = u + v;
+                    x[i + hs] = u - v;
+                }
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < kHeadDim; ++i) {
+            x[i] *= kLog2eTc / kHeadDim;        // (H q / sqrt d) . y / sqrt d = (H q) . y / d
+            amax = fmaxf(amax, fabsf(x[i]));
+        }
+        const int ex = amax > 0.f ? max(-100, min(100, ilogbf(amax))) : 0;
+        const float pre = pow2i(12 - ex);
+        rowfac = pow2i(ex - 12);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            uint32_t hw[16], lw[16];
+#pragma unroll
+            for (int w = 0; w < 16; ++w) {
+                const int k0 = 32 * c + 2 * w;
+                const float q0 = x[perm_k<F::GB>(k0)] * pre, q1 = x[perm_k<F::GB>(k0 + 1)] * pre;
+                hw[w] = split_hi_lo<true>(q0, q1, true);
+                lw[w] = split_hi_lo<true>(q0, q1, false);
+            }
+            tmem_st16(t_lane + kPfColQ + 16 * c, hw);
+            tmem_st16(t_lane + kPfColQ + 64 + 16 * c, lw);
+        }
+    }
+
+    const uint64_t desc_k = smem_desc(kdeq, kLbo, 128);
+    const uint64_t desc_v = smem_desc(vdeq, kLbo, 128);
+    const float kinv = F::kDequant;
+    float m_run = -CUDART_INF_F, l_run = 0.f;
+    int ev = 0;                                   // running V-scale exponent (biased), CTA-uniform
+    float vn = 1.f;                               // 2^(127 - ev)
+    bool aborted = false;
+
+    for (int t = 0; t < ntiles; ++t) {
+        const int stage = t % kStages;
+        uint8_t* st = ring + stage * F::kStage;
+        const int tok0 = t * kTile;
+        bool ok = mbar_wait_sleep(&full[stage], (uint32_t)((t / kStages) & 1), kPollsTc);
+        // PV(t - 1) has drained: the dequantised V, the P' columns and O are free
+        if (t > 0) ok = ok && mbar_wait_sleep(bar_o, (uint32_t)((t - 1) & 1), kPollsTc);
+        tc_fence_after();
+        if (!ok) atomicOr(&s_flag[0], 1);
+
+        // 1. token tid's K row and dimension tid's V column -> f16 B operands
+        {
+            const int pg = tid >> a.lp, row = tid & (P - 1);
+            const uint8_t* kblk = st + pg * 2 * a.block_bytes;
+            const uint8_t* vblk = kblk + a.block_bytes;
+            k_row_unpack<BITS>(kblk + row * F::CB, k_swizzle<BITS>(row), [&](int c, const uint32_t* o) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    *reinterpret_cast<uint4*>(kdeq + pf_b_offset(tid, 2 * (c + 4 * i))) =
+                        make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+            });
+            v_col_unpack<BITS>(st + a.block_bytes, 2 * a.block_bytes, a.lp, tid,
+                               [&](int c, const uint32_t* o) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    *reinterpret_cast<uint4*>(vdeq + pf_b_offset(tid, 2 * (c + 4 * i))) =
+                        make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+            });
+            const bool live = tok0 + tid < nkeys;
+            s_ks[tid] = live ? reinterpret_cast<const float*>(kblk + P * F::CB)[row] * kinv : 0.f;
+            s_vs[tid] = live ? reinterpret_cast<const float*>(vblk + P * F::CB)[row] * kinv : 0.f;
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();                          // also: the stage is consumed
+        if (s_flag[0]) { aborted = true; break; }
+        if (warp == 0 && t + kStages < ntiles)
+            issue_tile_tc(st, &full[stage], a, pt + (((t + kStages) * kTile) >> a.lp), kvh,
+                          min(kTile, nkeys - (t + kStages) * kTile), lane);
+
+        // 2. S = Q' K^T (hi, then lo)
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                umma_f16_ts(tmem + kPfColS, tmem + kPfColQ + 8 * j, desc_k + ((2 * j * kLbo) >> 4),
+                            kIdesc, j > 0);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                umma_f16_ts(tmem + kPfColS, tmem + kPfColQ + 64 + 8 * j,
+                            desc_k + ((2 * j * kLbo) >> 4), kIdesc, 1u);
+            umma_commit(bar_s);
+        }
+
+        // the tile's largest V scale (every thread reads all of them: uniform)
+        unsigned vmaxb = 0;
+#pragma unroll 8
+        for (int i = 0; i < kTile; ++i) vmaxb = max(vmaxb, __float_as_uint(s_vs[i]));
+        const int ev_new = max(ev, (int)(vmaxb >> 23));
+
+        ok = mbar_wait_sleep(bar_s, (uint32_t)(t & 1), kPollsTc);
+        tc_fence_after();
+        if (!ok) atomicOr(&s_flag[0], 1);
+
+        // 3a. this row's maximum over the tile
+        const float sfac = rowfac;
+        float tmax = -CUDART_INF_F;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            uint32_t v[32];
+            tmem_ld16(t_lane + kPfColS + 32 * c, v);
+            tmem_ld16(t_lane + kPfColS + 32 * c + 16, v + 16);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int key = 32 * c + i;
+                const float xs = __uint_as_float(v[i]) * (s_ks[key] * sfac);
+                tmax = fmaxf(tmax, tok0 + key <= lim ? xs : -CUDART_INF_F);
+            }
+        }
+        // rescale O (this warp's rows) when a row gains more than 2^8 or the
+        // V-scale exponent grows
+        const float mn = fmaxf(m_run, tmax);
+        const bool grow = mn > m_run + kLazyTc;
+        const float m_use = grow ? mn : m_run;
+        const float alpha = (grow && m_run != -CUDART_INF_F) ? fast_exp2(m_run - mn) : 1.f;
+        const float av = pow2i(ev - ev_new);
+        if (t > 0 && (__any_sync(kFull, alpha != 1.f) || ev_new != ev)) {
+            const float f = alpha * av;
+#pragma unroll
+            for (int c = 0; c < 128; c += 16) {
+                uint32_t ov[16];
+                tmem_ld16(t_lane + kPfColO + c, ov);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
+                tmem_st16(t_lane + kPfColO + c, ov);
+            }
+        }
+        l_run *= alpha;
+        m_run = m_use;
+        ev = ev_new;
+        vn = pow2i(127 - ev);
+
+        // 3b. weights of this row -> P' (hi, lo), keys in the V unpacker's order
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            uint32_t v[32];
+            tmem_ld16(t_lane + kPfColS + 32 * c, v);
+            tmem_ld16(t_lane + kPfColS + 32 * c + 16, v + 16);
+            tmem_wait_ld();
+            float pv[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int key = 32 * c + i;
+                const float xs = __uint_as_float(v[i]) * (s_ks[key] * sfac);
+                const float p = tok0 + key <= lim ? fast_exp2(xs - m_run) : 0.f;
+                l_run += p;
+                pv[i] = p * (s_vs[key] * vn);
+            }
+            uint32_t hw[16], lw[16];
+#pragma unroll
+            for (int w = 0; w < 16; ++w) {
+                const float p0 = pv[perm_k<F::GB>(2 * w)], p1 = pv[perm_k<F::GB>(2 * w + 1)];
+                hw[w] = split_hi_lo<true>(p0, p1, true);
+                lw[w] = split_hi_lo<true>(p0, p1, false);
+            }
+            tmem_st16(t_lane + kPfColP + 16 * c, hw);
+            tmem_st16(t_lane + kPfColP + 64 + 16 * c, lw);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+
+        // 4. O += P' V (hi, then lo)
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                umma_f16_ts(tmem + kPfColO, tmem + kPfColP + 8 * j, desc_v + ((2 * j * kLbo) >> 4),
+                            kIdesc, (t > 0 || j > 0) ? 1u : 0u);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                umma_f16_ts(tmem + kPfColO, tmem + kPfColP + 64 + 8 * j,
+                            desc_v + ((2 * j * kLbo) >> 4), kIdesc, 1u);
+            umma_commit(bar_o);
+        }
+    }
+
+    // ---- epilogue: normalise, rotate back, write this row
+    bool ok = !aborted && ntiles > 0 &&
+              mbar_wait_sleep(bar_o, (uint32_t)((ntiles - 1) & 1), kPollsTc);
+    tc_fence_after();
+    ok = __syncthreads_and(ok);
+    if (ok) {
+        float x[kHeadDim];
+#pragma unroll
+        for (int c = 0; c < kHeadDim; c += 16) {
+            uint32_t ov[16];
+            tmem_ld16(t_lane + kPfColO + c, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) x[c + i] = __uint_as_float(ov[i]);
+        }
+        const float inv = (l_run > 0.f ? 1.f / l_run : 0.f) * pow2i(ev - 127) *
+                          0.08838834764831845f;     // V-scale exponent back, 1 / sqrt d
+#pragma unroll
+        for (int hs = 1; hs < kHeadDim; hs <<= 1)
+#pragma unroll
+            for (int i = 0; i < kHeadDim; ++i)
+                if (!(i & hs)) {
+                    const float u = x[i], v = x[i + hs];
+                    x[i] = u + v;
+                    x[i + hs] = u - v;
+                }
+        if (row_ok) {
+            float4* dst = reinterpret_cast<float4*>(
+                a.out + (((int64_t)b * a.q_len + tq) * a.num_q_heads + h) * kHeadDim);
+#pragma unroll
+            for (int c = 0; c < kHeadDim / 4; ++c)
+                dst[c] = make_float4(x[4 * c] * inv, x[4 * c + 1] * inv, x[4 * c + 2] * inv,
+                                     x[4 * c + 3] * inv);
+        }
+    } else if (tid == 0 && ntiles > 0) {
+        report_error(a.err, TQ_ERR_TIMEOUT, kErrWaitTile);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kPfTmemCols);
+    }
+}
+
+template <int BITS>
+cudaError_t launch_prefill(const TcArgs& a, int batch, cudaStream_t stream)
+{
+    const size_t smem = kPfRing + (size_t)kStages * TcFmt<BITS>::kStage;
+    static int configured = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 31 || !(configured & (1 << dev))) {
+        e = cudaFuncSetAttribute(k_prefill_tc<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+        if (e != cudaSuccess) return e;
+        if (dev < 31) configured |= 1 << dev;
+    }
+    const dim3 grid((unsigned)((a.G + kPfRows - 1) / kPfRows), (unsigned)a.num_kv_heads,
+                    (unsigned)batch);
+    k_prefill_tc<BITS><<<grid, kTcThreads, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 // Query rows of one tensor-core CTA: 4, 8 or 16.  Up to 4 rows, 2-, 4- and
@@ -1547,6 +1948,13 @@ int decode_tc_rows(int format, int G)
 {
     (void)format;
     return G <= 4 ? 4 : (G <= 8 ? 8 : 16);
+}
+
+// The query-major kernel takes 128 or more rows per kv head of a turbo format;
+// it writes its rows directly (no splits, no workspace).
+bool decode_uses_prefill(int format, int G)
+{
+    return format != TQ_FP8 && format != 16 && G >= kPfRows;
 }
 
 cudaError_t launch_decode_tc(const void* q, const tq_cache& c, int64_t block_bytes,
@@ -1569,6 +1977,20 @@ cudaError_t launch_decode_tc(const void* q, const tq_cache& c, int64_t block_byt
     a.group = num_q_heads / c.num_kv_heads;
     a.q_len = q_len;
     a.G = q_len * a.group;
+    a.page_size = c.page_size;
+    a.lp = c.page_size == 16 ? 4 : (c.page_size == 32 ? 5 : 6);
+    a.max_seq_len = max_seq_len;
+    // 128 or more rows per kv head (prefill chunks, long verify windows),
+    // turbo formats: the query-major kernel, one CTA per 128 rows
+    if (decode_uses_prefill(c.format, a.G)) {
+        switch (c.format) {
+        case 2: return launch_prefill<2>(a, batch, stream);
+        case 3: return launch_prefill<3>(a, batch, stream);
+        case 4: return launch_prefill<4>(a, batch, stream);
+        case 8: return launch_prefill<8>(a, batch, stream);
+        default: return cudaErrorInvalidValue;
+        }
+    }
     const int rows = decode_tc_rows(c.format, a.G);
     a.R = (a.G + rows - 1) / rows;
     a.page_size = c.page_size;

@@ -238,11 +238,15 @@ def test_causal_last_split_fully_masked_rows(q_len, lens):
     (16, 96, (2200, 500)),       # bf16 cache: 8-row groups
     (2, 256, (4096, 2400)),      # 1024 rows; a chunk at the end of two splits
     (FP8, 48, (2100, 60)),
+    (8, 32, (1500, 40)),         # exactly 128 rows: one query-major CTA per kv head
+    (4, 33, (900, 2049)),        # 132 rows: a second row block of 4 rows
+    (3, 40, (129, 3000)),        # 160 rows, a context of 89 tokens before the chunk
 ])
 def test_chunked_prefill_over_quantised_pages(fmt, q_len, lens):
     """A chunk of q_len prefill tokens, appended first, attends causally over
     the cache: row t sees keys j <= seq_len - q_len + t.  Every row of every
-    chunk against the oracle."""
+    chunk against the oracle (128 or more rows per kv head take the
+    query-major kernel for turbo formats)."""
     w = small(fmt, q_len=q_len, seq_lens=lens)
     cache = gpu_fill(w, fmt)
     check_close(gpu_decode(w, fmt, cache), oracle_decode(w, fmt, np.arange(len(lens))),
