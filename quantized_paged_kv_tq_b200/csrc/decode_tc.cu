@@ -1558,20 +1558,22 @@ cudaError_t launch_i8(const TcArgs& a, dim3 grid, cudaStream_t stream)
 // Query-major kernel for long verify windows and prefill chunks (turbo
 // formats, G = q_len x GQA >= 128 rows per kv head).
 //
-// One CTA (128 threads) owns 128 query rows of one (sequence, kv head) and
+// One CTA (256 threads) owns 128 query rows of one (sequence, kv head) and
 // walks every key tile its rows may see (causal), so each K/V tile is
 // dequantised once for 128 rows instead of once per 16-row group:
-//   1. token t unpacks its K row, and dimension t its V column, into exact
-//      f16 integers in shared memory, in the canonical K-major layout (8x8
-//      core matrices) of the MMA's B operand; the tile's K and V scales go
-//      to shared memory too.
+//   1. thread t < 128 unpacks token t's K row, thread 128 + d dimension d's V
+//      column, into exact f16 integers in shared memory, in the canonical
+//      K-major layout (8x8 core matrices) of the MMA's B operand; the tile's
+//      K and V scales go to shared memory too.
 //   2. one thread issues S[128 rows][128 keys] = Q' K^T: A = Q' in tensor
 //      memory (the rotated query, prescaled per row, split into f16 hi and
 //      lo parts: two MMA chains into one fp32 accumulator).
-//   3. thread r owns row r: it reads its scores (twice: the row maximum,
-//      then the weights), scales them by s_k / L and the row factor, masks
-//      keys beyond its causal limit, and runs an online softmax with a lazy
-//      maximum (a warp rescales its rows of O only when one of them gains
+//   3. two threads own row r (warps w and w + 4 reach the same tensor-memory
+//      lanes), one per half of the keys: each reads its scores (twice: the
+//      row maximum, exchanged through shared memory, then the weights),
+//      scales them by s_k / L and the row factor, masks keys beyond the
+//      row's causal limit, and runs an online softmax with a lazy maximum (a
+//      warp rescales its half of its rows of O only when one of them gains
 //      more than 2^8).  P' = p s_v / L 2^(127 - ev), split hi/lo in f16, goes
 //      to tensor memory as the A operand of the PV product (keys in the V
 //      unpacker's pair order).
@@ -1581,12 +1583,16 @@ cudaError_t launch_i8(const TcArgs& a, dim3 grid, cudaStream_t stream)
 // Tensor memory: Q' hi/lo 128 columns, S 128, O 128, P' hi/lo 128.
 // ===================================================================
 constexpr int kPfRows = 128;
+constexpr int kPfThreads = 256;
 constexpr uint32_t kPfColQ = 0, kPfColS = 128, kPfColO = 256, kPfColP = 384;
 constexpr uint32_t kPfTmemCols = 512;
 // shared memory (bytes from the start)
 constexpr int kPfKs = 128;          // [128] K scales of the tile, / L
 constexpr int kPfVs = 640;          // [128] V scales of the tile, / L
-constexpr int kPfKdeq = 2048;       // [128 keys x 128 dims] f16, B of S
+constexpr int kPfRowfac = 1152;     // [128] row factors
+constexpr int kPfPmax = 1664;       // [2][128] row maxima of the two key halves
+constexpr int kPfL = 2688;          // [2][128] row sums of the two key halves
+constexpr int kPfKdeq = 4096;       // [128 keys x 128 dims] f16, B of S
 constexpr int kPfVdeq = kPfKdeq + 32768;   // [128 dims x 128 keys] f16, B of O
 constexpr int kPfRing = kPfVdeq + 32768;   // [kStages] tile stages
 
@@ -1599,7 +1605,7 @@ __device__ __forceinline__ int pf_b_offset(int n, int k)
 }
 
 template <int BITS>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kPfThreads, 1)
 k_prefill_tc(const TcArgs a)
 {
     using F = TcFmt<BITS>;
@@ -1615,6 +1621,9 @@ k_prefill_tc(const TcArgs a)
     int* s_flag = reinterpret_cast<int*>(smem + 68);
     float* s_ks = reinterpret_cast<float*>(smem + kPfKs);
     float* s_vs = reinterpret_cast<float*>(smem + kPfVs);
+    float* s_rowfac = reinterpret_cast<float*>(smem + kPfRowfac);
+    float* s_pmax = reinterpret_cast<float*>(smem + kPfPmax);
+    float* s_lsum = reinterpret_cast<float*>(smem + kPfL);
     uint8_t* kdeq = smem + kPfKdeq;
     uint8_t* vdeq = smem + kPfVdeq;
     uint8_t* ring = smem + kPfRing;
@@ -1627,8 +1636,10 @@ k_prefill_tc(const TcArgs a)
         return;
     }
     const int P = a.page_size;
-    // this thread's row, its causal limit; the block's last visible key
-    const int R = rb * kPfRows + tid;
+    // this thread's row (tensor-memory lane) and half of the keys; the row's
+    // causal limit; the block's last visible key
+    const int r = 32 * (warp & 3) + lane, hk = warp >> 2;
+    const int R = rb * kPfRows + r;
     const bool row_ok = R < a.G;
     const int tq = row_ok ? R / a.group : 0;
     const int h = kvh * a.group + (R - tq * a.group);
@@ -1653,17 +1664,17 @@ k_prefill_tc(const TcArgs a)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    const uint32_t t_lane = tmem + ((uint32_t)(32 * warp) << 16);
+    const uint32_t t_lane = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
 
     if (warp == 0)
         for (int s = 0; s < kStages && s < ntiles; ++s)
             issue_tile_tc(ring + s * F::kStage, &full[s], a, pt + ((s * kTile) >> a.lp), kvh,
                           min(kTile, nkeys - s * kTile), lane);
 
-    // ---- Q' of this row: rotate (128-point FWHT in registers), log2 scale,
-    // power-of-two prescale, f16 hi + lo in the K unpacker's dimension order
-    float rowfac = 1.f;
-    {
+    // ---- Q' of this row (first half of the threads): rotate (128-point
+    // FWHT in registers), log2 scale, power-of-two prescale, f16 hi + lo in
+    // the K unpacker's dimension order
+    if (hk == 0) {
         float x[kHeadDim];
         if (row_ok) {
             const uint4* src = reinterpret_cast<const uint4*>(
@@ -1699,7 +1710,7 @@ k_prefill_tc(const TcArgs a)
         }
         const int ex = amax > 0.f ? max(-100, min(100, ilogbf(amax))) : 0;
         const float pre = pow2i(12 - ex);
-        rowfac = pow2i(ex - 12);
+        s_rowfac[r] = pow2i(ex - 12);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             uint32_t hw[16], lw[16];
@@ -1713,8 +1724,11 @@ k_prefill_tc(const TcArgs a)
             tmem_st16(t_lane + kPfColQ + 16 * c, hw);
             tmem_st16(t_lane + kPfColQ + 64 + 16 * c, lw);
         }
+        tmem_wait_st();                           // complete before the first S product
     }
 
+    __syncthreads();                              // row factors
+    const float rowfac = s_rowfac[r];
     const uint64_t desc_k = smem_desc(kdeq, kLbo, 128);
     const uint64_t desc_v = smem_desc(vdeq, kLbo, 128);
     const float kinv = F::kDequant;
@@ -1733,27 +1747,33 @@ k_prefill_tc(const TcArgs a)
         tc_fence_after();
         if (!ok) atomicOr(&s_flag[0], 1);
 
-        // 1. token tid's K row and dimension tid's V column -> f16 B operands
+        // 1. token u's K row (threads u < 128) or dimension u's V column
+        // (threads 128 + u) -> f16 B operands; token u's K or V scale
         {
-            const int pg = tid >> a.lp, row = tid & (P - 1);
+            const int u = tid & (kTile - 1);
+            const int pg = u >> a.lp, row = u & (P - 1);
             const uint8_t* kblk = st + pg * 2 * a.block_bytes;
             const uint8_t* vblk = kblk + a.block_bytes;
-            k_row_unpack<BITS>(kblk + row * F::CB, k_swizzle<BITS>(row), [&](int c, const uint32_t* o) {
+            const bool live = tok0 + u < nkeys;
+            if (hk == 0) {
+                k_row_unpack<BITS>(kblk + row * F::CB, k_swizzle<BITS>(row),
+                                   [&](int c, const uint32_t* o) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    *reinterpret_cast<uint4*>(kdeq + pf_b_offset(tid, 2 * (c + 4 * i))) =
-                        make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-            });
-            v_col_unpack<BITS>(st + a.block_bytes, 2 * a.block_bytes, a.lp, tid,
-                               [&](int c, const uint32_t* o) {
+                    for (int i = 0; i < 4; ++i)
+                        *reinterpret_cast<uint4*>(kdeq + pf_b_offset(u, 2 * (c + 4 * i))) =
+                            make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+                });
+                s_ks[u] = live ? reinterpret_cast<const float*>(kblk + P * F::CB)[row] * kinv : 0.f;
+            } else {
+                v_col_unpack<BITS>(st + a.block_bytes, 2 * a.block_bytes, a.lp, u,
+                                   [&](int c, const uint32_t* o) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    *reinterpret_cast<uint4*>(vdeq + pf_b_offset(tid, 2 * (c + 4 * i))) =
-                        make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-            });
-            const bool live = tok0 + tid < nkeys;
-            s_ks[tid] = live ? reinterpret_cast<const float*>(kblk + P * F::CB)[row] * kinv : 0.f;
-            s_vs[tid] = live ? reinterpret_cast<const float*>(vblk + P * F::CB)[row] * kinv : 0.f;
+                    for (int i = 0; i < 4; ++i)
+                        *reinterpret_cast<uint4*>(vdeq + pf_b_offset(u, 2 * (c + 4 * i))) =
+                            make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+                });
+                s_vs[u] = live ? reinterpret_cast<const float*>(vblk + P * F::CB)[row] * kinv : 0.f;
+            }
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -1780,29 +1800,42 @@ k_prefill_tc(const TcArgs a)
         // the tile's largest V scale (every thread reads all of them: uniform)
         unsigned vmaxb = 0;
 #pragma unroll 8
-        for (int i = 0; i < kTile; ++i) vmaxb = max(vmaxb, __float_as_uint(s_vs[i]));
+        for (int i = 0; i < kTile; i += 4) {
+            const uint4 x = *reinterpret_cast<const uint4*>(s_vs + i);
+            vmaxb = max(max(vmaxb, max(x.x, x.y)), max(x.z, x.w));
+        }
         const int ev_new = max(ev, (int)(vmaxb >> 23));
 
         ok = mbar_wait_sleep(bar_s, (uint32_t)(t & 1), kPollsTc);
         tc_fence_after();
         if (!ok) atomicOr(&s_flag[0], 1);
 
-        // 3a. this row's maximum over the tile
-        const float sfac = rowfac;
-        float tmax = -CUDART_INF_F;
+        // 3a. this row's maximum over the tile: each thread its half of the
+        // keys (the row factor is a positive constant: applied after)
+        float hmax = -CUDART_INF_F;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * hk + cc;
             uint32_t v[32];
             tmem_ld16(t_lane + kPfColS + 32 * c, v);
             tmem_ld16(t_lane + kPfColS + 32 * c + 16, v + 16);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int key = 32 * c + i;
-                const float xs = __uint_as_float(v[i]) * (s_ks[key] * sfac);
-                tmax = fmaxf(tmax, tok0 + key <= lim ? xs : -CUDART_INF_F);
+            for (int i = 0; i < 32; i += 4) {
+                const float4 ks4 = *reinterpret_cast<const float4*>(s_ks + 32 * c + i);
+                const float kk[4] = {ks4.x, ks4.y, ks4.z, ks4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int key = 32 * c + i + e;
+                    const float xs = __uint_as_float(v[i + e]) * kk[e];
+                    hmax = fmaxf(hmax, tok0 + key <= lim ? xs : -CUDART_INF_F);
+                }
             }
         }
+        s_pmax[hk * kPfRows + r] = hmax;
+        __syncthreads();
+        const float sfac = rowfac;
+        const float tmax = fmaxf(s_pmax[r], s_pmax[kPfRows + r]) * sfac;
         // rescale O (this warp's rows) when a row gains more than 2^8 or the
         // V-scale exponent grows
         const float mn = fmaxf(m_run, tmax);
@@ -1813,7 +1846,7 @@ k_prefill_tc(const TcArgs a)
         if (t > 0 && (__any_sync(kFull, alpha != 1.f) || ev_new != ev)) {
             const float f = alpha * av;
 #pragma unroll
-            for (int c = 0; c < 128; c += 16) {
+            for (int c = 64 * hk; c < 64 * hk + 64; c += 16) {
                 uint32_t ov[16];
                 tmem_ld16(t_lane + kPfColO + c, ov);
                 tmem_wait_ld();
@@ -1827,21 +1860,30 @@ k_prefill_tc(const TcArgs a)
         ev = ev_new;
         vn = pow2i(127 - ev);
 
-        // 3b. weights of this row -> P' (hi, lo), keys in the V unpacker's order
+        // 3b. weights of this row's half of the keys -> P' (hi, lo), keys in
+        // the V unpacker's order
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * hk + cc;
             uint32_t v[32];
             tmem_ld16(t_lane + kPfColS + 32 * c, v);
             tmem_ld16(t_lane + kPfColS + 32 * c + 16, v + 16);
             tmem_wait_ld();
             float pv[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int key = 32 * c + i;
-                const float xs = __uint_as_float(v[i]) * (s_ks[key] * sfac);
-                const float p = tok0 + key <= lim ? fast_exp2(xs - m_run) : 0.f;
-                l_run += p;
-                pv[i] = p * (s_vs[key] * vn);
+            for (int i = 0; i < 32; i += 4) {
+                const float4 ks4 = *reinterpret_cast<const float4*>(s_ks + 32 * c + i);
+                const float4 vs4 = *reinterpret_cast<const float4*>(s_vs + 32 * c + i);
+                const float kk[4] = {ks4.x, ks4.y, ks4.z, ks4.w};
+                const float vv[4] = {vs4.x, vs4.y, vs4.z, vs4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int key = 32 * c + i + e;
+                    const float xs = __uint_as_float(v[i + e]) * (kk[e] * sfac);
+                    const float p = tok0 + key <= lim ? fast_exp2(xs - m_run) : 0.f;
+                    l_run += p;
+                    pv[i + e] = p * (vv[e] * vn);
+                }
             }
             uint32_t hw[16], lw[16];
 #pragma unroll
@@ -1872,12 +1914,15 @@ k_prefill_tc(const TcArgs a)
         }
     }
 
-    // ---- epilogue: normalise, rotate back, write this row
+    // ---- epilogue (first half of the threads): normalise, rotate back,
+    // write this row
     bool ok = !aborted && ntiles > 0 &&
               mbar_wait_sleep(bar_o, (uint32_t)((ntiles - 1) & 1), kPollsTc);
     tc_fence_after();
+    s_lsum[hk * kPfRows + r] = l_run;
     ok = __syncthreads_and(ok);
-    if (ok) {
+    if (ok && hk == 0) {
+        l_run = s_lsum[r] + s_lsum[kPfRows + r];
         float x[kHeadDim];
 #pragma unroll
         for (int c = 0; c < kHeadDim; c += 16) {
@@ -1933,7 +1978,7 @@ cudaError_t launch_prefill(const TcArgs& a, int batch, cudaStream_t stream)
     }
     const dim3 grid((unsigned)((a.G + kPfRows - 1) / kPfRows), (unsigned)a.num_kv_heads,
                     (unsigned)batch);
-    k_prefill_tc<BITS><<<grid, kTcThreads, smem, stream>>>(a);
+    k_prefill_tc<BITS><<<grid, kPfThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
