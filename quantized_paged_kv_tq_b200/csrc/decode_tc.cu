@@ -1593,8 +1593,8 @@ constexpr int kPfRowfac = 1152;     // [128] row factors
 constexpr int kPfPmax = 1664;       // [2][128] row maxima of the two key halves
 constexpr int kPfL = 2688;          // [2][128] row sums of the two key halves
 constexpr int kPfKdeq = 4096;       // [128 keys x 128 dims] f16, B of S
-constexpr int kPfVdeq = kPfKdeq + 32768;   // [128 dims x 128 keys] f16, B of O
-constexpr int kPfRing = kPfVdeq + 32768;   // [kStages] tile stages
+constexpr int kPfVdeq = kPfKdeq + 32768;   // [2][128 dims x 128 keys] f16, B of O, by tile parity
+constexpr int kPfRing = kPfVdeq + 2 * 32768;   // [kStages] tile stages
 
 // K-major core-matrix offset (bytes) of element (n, k) of a [128 x 128] f16
 // B operand: 8x8 core matrices of 128 bytes, N-adjacent ones 128 bytes
@@ -1625,7 +1625,7 @@ k_prefill_tc(const TcArgs a)
     float* s_pmax = reinterpret_cast<float*>(smem + kPfPmax);
     float* s_lsum = reinterpret_cast<float*>(smem + kPfL);
     uint8_t* kdeq = smem + kPfKdeq;
-    uint8_t* vdeq = smem + kPfVdeq;
+    uint8_t* vdeq0 = smem + kPfVdeq;
     uint8_t* ring = smem + kPfRing;
 
     const int rb = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -1730,7 +1730,7 @@ k_prefill_tc(const TcArgs a)
     __syncthreads();                              // row factors
     const float rowfac = s_rowfac[r];
     const uint64_t desc_k = smem_desc(kdeq, kLbo, 128);
-    const uint64_t desc_v = smem_desc(vdeq, kLbo, 128);
+    const uint64_t desc_v0 = smem_desc(vdeq0, kLbo, 128);
     const float kinv = F::kDequant;
     float m_run = -CUDART_INF_F, l_run = 0.f;
     int ev = 0;                                   // running V-scale exponent (biased), CTA-uniform
@@ -1741,9 +1741,10 @@ k_prefill_tc(const TcArgs a)
         const int stage = t % kStages;
         uint8_t* st = ring + stage * F::kStage;
         const int tok0 = t * kTile;
+        uint8_t* vdeq = vdeq0 + (t & 1) * 32768;
+        // the V buffer of this tile was last read by PV(t - 2), which drained
+        // before tile t - 1's weights were written
         bool ok = mbar_wait_sleep(&full[stage], (uint32_t)((t / kStages) & 1), kPollsTc);
-        // PV(t - 1) has drained: the dequantised V, the P' columns and O are free
-        if (t > 0) ok = ok && mbar_wait_sleep(bar_o, (uint32_t)((t - 1) & 1), kPollsTc);
         tc_fence_after();
         if (!ok) atomicOr(&s_flag[0], 1);
 
@@ -1833,6 +1834,13 @@ k_prefill_tc(const TcArgs a)
             }
         }
         s_pmax[hk * kPfRows + r] = hmax;
+        // PV(t - 1) has drained (it ran under this tile's unpack, S product
+        // and maximum): O and the P' columns are free
+        if (t > 0) {
+            ok = mbar_wait_sleep(bar_o, (uint32_t)((t - 1) & 1), kPollsTc);
+            tc_fence_after();
+            if (!ok) atomicOr(&s_flag[0], 1);
+        }
         __syncthreads();
         const float sfac = rowfac;
         const float tmax = fmaxf(s_pmax[r], s_pmax[kPfRows + r]) * sfac;
@@ -1902,6 +1910,7 @@ k_prefill_tc(const TcArgs a)
         // 4. O += P' V (hi, then lo)
         if (tid == 0) {
             tc_fence_after();
+            const uint64_t desc_v = desc_v0 + (uint64_t)(((t & 1) * 32768) >> 4);
 #pragma unroll
             for (int j = 0; j < 8; ++j)
                 umma_f16_ts(tmem + kPfColO, tmem + kPfColP + 8 * j, desc_v + ((2 * j * kLbo) >> 4),
