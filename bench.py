@@ -665,8 +665,7 @@ def extra_rows(tq, dev, peak, timed):
             torch.bfloat16).to(dev)
 
     # ---- prefill chunk
-    w = W.custom(batch=4, num_q_heads=32, num_kv_heads=8, page_size=16, q_len=256,
-                 seq_lens=(4096,) * 4, fmt=4, seed=9)
+    w = W.make("prefill256")
     cache = tq.Cache(4, w.num_pages, w.num_kv_heads, w.page_size, device=dev)
     for slots, k, v in w.iter_fill(1 << 16):
         tq.tq_quantize_append(d_bf16(k), d_bf16(v), torch.from_numpy(slots.astype(np.int64)).to(dev),
@@ -692,15 +691,14 @@ def extra_rows(tq, dev, peak, timed):
     pairs *= w.num_kv_heads
     flops = pairs * 4 * w.head_dim                      # QK and PV, 2 flops per MAC
     uniq = int(w.seq_lens.sum()) * w.num_kv_heads * 2 * W.row_bytes(4)
-    rows.append({"workload": "prefill chunk: batch 4 x 4096-token context, the last 256 tokens "
+    rows.append({"workload": "prefill256: batch 4 x 4096-token context, the last 256 tokens "
                              "a prefill chunk, 32 q / 8 kv heads, page 16, turbo4",
                  "kernel": decode_kernel_label(4, G), "rows_per_kv_head": G,
                  "decode_us": ms * 1e3, "decode_us_min": ms_min * 1e3,
                  "chunk_tokens_per_s": w.batch * w.q_len / (ms * 1e-3),
                  "tflops": flops / (ms * 1e-3) / 1e12, "flops": flops,
                  "unique_kv_bytes": uniq, "unique_frac_of_hbm": uniq / (ms * 1e-3) / 1e9 / peak,
-                 "l2": "flushed before every timed launch; the 16-row groups re-read a kv "
-                       "head's pages, mostly from L2"})
+                 "l2": "flushed before every timed launch"})
     del cache, ws, q, out
     torch.cuda.empty_cache()
 

@@ -240,6 +240,10 @@ def make(name: str) -> Workload:
                 sequences 0-15 share a 2048-token prefix through the same
                 physical pages, private suffixes of 256-4096 tokens, page 16,
                 turbo4, 4 outlier channels, seed 4.
+    prefill256  batch 4, 32 / 8, context 4096 whose last 256 tokens are a
+                prefill chunk (q_len 256: 1024 query rows per kv head,
+                causal), page 16, turbo4, 2 key and 1 value outlier channels,
+                seed 9.
     """
     if name == "tiny":
         w = Workload(name, 1, 4, 1, 16, 1, (4,), 0, k_outliers=2)
@@ -264,6 +268,10 @@ def make(name: str) -> Workload:
                      shared_prefix_seqs=16, shared_prefix_tokens=2048)
         w.seq_lens = (2048 + np.random.default_rng([4, _S_LENS]).integers(
             256, 4096, size=32, endpoint=True)).astype(np.int32)
+    elif name == "prefill256":
+        w = Workload(name, 4, 32, 8, 16, 256, (4,), 9, k_outliers=2, v_outliers=1,
+                     permute_pages=True)
+        w.seq_lens = np.full(4, 4096, np.int32)
     else:
         raise KeyError(name)
     return _finish(w)
@@ -285,4 +293,4 @@ def custom(name="custom", batch=2, num_q_heads=8, num_kv_heads=2, page_size=16,
     return _finish(w)
 
 
-ALL = ("tiny", "batch8", "cbatch64", "target64x8k", "long128k", "specverify")
+ALL = ("tiny", "batch8", "cbatch64", "target64x8k", "long128k", "specverify", "prefill256")
