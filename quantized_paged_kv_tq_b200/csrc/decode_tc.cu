@@ -91,6 +91,23 @@ struct TcFmt {
     static constexpr int kStage = 2 * kTile * (CB + 4);   // K and V blocks of one tile
 };
 
+// Shared-memory header of the f16 kernel (byte offsets): barriers at 0,
+// TMEM address and flags at 64, per-warp row reductions with a stride of kRS
+// rows, the split's page ids, then the operands.  Up to 8 rows the header
+// is 1 KB, so that three CTAs with two 33 KB stages of 8-bit codes fit the
+// 228 KB of an SM.
+template <int RG>
+struct TcHdr {
+    static constexpr int kRS = RG <= 8 ? 8 : 16;
+    static constexpr int kRed = 128;                   // float [4][kRS]
+    static constexpr int kRedv = kRed + 16 * kRS;      // unsigned [4]
+    static constexpr int kRowfac = kRedv + 16;         // float [kRS]
+    static constexpr int kL = kRowfac + 4 * kRS;       // float [4][kRS]
+    static constexpr int kPid = RG <= 8 ? 512 : 1024;  // int [128]
+    static constexpr int kBytes = kPid + 512;
+    static_assert(RG <= kRS && kL + 16 * kRS <= kPid, "header overlap");
+};
+
 // Two E4M3 codes (low byte first) -> f16x2 (exact: every E4M3 value is an f16)
 __device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t two)
 {
@@ -418,7 +435,7 @@ __device__ __forceinline__ void load_split_pids(int* s_pid, const TcArgs& a, int
 
 // Split epilogue shared by the tensor-core kernels.  sO: the split's
 // un-normalised output rows [RG][128] (rotated domain); s_l: per-warp partial
-// row sums [4][16]; m_run: row maxima (log2 units).  A split that is the whole
+// row sums [4][LS]; m_run: row maxima (log2 units).  A split that is the whole
 // sequence normalises, rotates back and writes; otherwise the partial goes to
 // the workspace and the last split CTA of the unit (atomic ticket) merges;
 // `unit` indexes the (sequence, kv head, row group) in the workspace.
@@ -426,7 +443,7 @@ __device__ __forceinline__ void load_split_pids(int* s_pid, const TcArgs& a, int
 // is read from sO, s_l or m_run; a split of a longer sequence still records
 // an empty partial (m = -inf) and takes its ticket, so the unit's counter
 // wraps back to zero and the workspace stays usable for later calls.
-template <int RG, bool ROT = true>
+template <int RG, int LS, bool ROT = true>
 __device__ __forceinline__ void tc_finish(const TcArgs& a, const float* sO, const float* s_l,
                                           const float* m_run, int* s_flag, int b, int kvh, int rg,
                                           int split, int nsplit, int nrows, int warp, int lane,
@@ -441,7 +458,7 @@ __device__ __forceinline__ void tc_finish(const TcArgs& a, const float* sO, cons
             continue;
         }
         const float M = m_run[rr];
-        const float Lsum = s_l[rr] + s_l[16 + rr] + s_l[32 + rr] + s_l[48 + rr];
+        const float Lsum = s_l[rr] + s_l[LS + rr] + s_l[2 * LS + rr] + s_l[3 * LS + rr];
         float x[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) x[e] = sO[rr * kHeadDim + 4 * lane + e];
@@ -529,12 +546,13 @@ k_decode_tc(const TcArgs a)
     uint64_t* bar_o = bar_s + 1;
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + 64);
     int* s_flag = reinterpret_cast<int*>(smem + 68);                 // [0] abort, [1] ticket
-    float* s_red = reinterpret_cast<float*>(smem + 128);             // [4][16] row maxima
-    unsigned* s_redv = reinterpret_cast<unsigned*>(smem + 384);      // [4]
-    float* s_rowfac = reinterpret_cast<float*>(smem + 400);          // [16]
-    float* s_l = reinterpret_cast<float*>(smem + 464);               // [4][16]
-    int* s_pid = reinterpret_cast<int*>(smem + 1024);                // [128] split page ids
-    uint8_t* s_qb = smem + 1536;                                     // Q' operand
+    using H = TcHdr<RG>;
+    float* s_red = reinterpret_cast<float*>(smem + H::kRed);         // [4][kRS] row maxima
+    unsigned* s_redv = reinterpret_cast<unsigned*>(smem + H::kRedv); // [4]
+    float* s_rowfac = reinterpret_cast<float*>(smem + H::kRowfac);   // [kRS]
+    float* s_l = reinterpret_cast<float*>(smem + H::kL);             // [4][kRS]
+    int* s_pid = reinterpret_cast<int*>(smem + H::kPid);             // [128] split page ids
+    uint8_t* s_qb = smem + H::kBytes;                                // Q' operand
     uint8_t* s_pb = s_qb + 256 * NCOL;                               // P' operand / q staging
     uint8_t* ring = s_pb + 256 * NCOL;
 
@@ -738,7 +756,7 @@ k_decode_tc(const TcArgs a)
                 float v = sc[r];
 #pragma unroll
                 for (int m = 16; m >= 1; m >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, m));
-                if (lane == 0) s_red[warp * 16 + r] = v;
+                if (lane == 0) s_red[warp * H::kRS + r] = v;
             }
             const unsigned vb = __reduce_max_sync(kFull, __float_as_uint(vs));
             if (lane == 0) s_redv[warp] = vb;
@@ -752,8 +770,8 @@ k_decode_tc(const TcArgs a)
             float alpha[RG];
 #pragma unroll
             for (int r = 0; r < RG; ++r) {
-                const float tmax = fmaxf(fmaxf(s_red[r], s_red[16 + r]),
-                                         fmaxf(s_red[32 + r], s_red[48 + r]));
+                const float tmax = fmaxf(fmaxf(s_red[r], s_red[H::kRS + r]),
+                                         fmaxf(s_red[2 * H::kRS + r], s_red[3 * H::kRS + r]));
                 const float mn = fmaxf(m_run[r], tmax);
                 alpha[r] = mn == -CUDART_INF_F ? 1.f : fast_exp2(m_run[r] - mn);
                 m_run[r] = mn;
@@ -842,7 +860,7 @@ k_decode_tc(const TcArgs a)
             float l = l_run[r];
 #pragma unroll
             for (int m = 16; m >= 1; m >>= 1) l += __shfl_xor_sync(kFull, l, m);
-            if (lane == 0) s_l[warp * 16 + r] = l;
+            if (lane == 0) s_l[warp * H::kRS + r] = l;
         }
     } else if (tid == 0) {
         report_error(a.err, TQ_ERR_TIMEOUT, kErrWaitTile);
@@ -853,7 +871,7 @@ k_decode_tc(const TcArgs a)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
-    tc_finish<RG, !FP8>(a, sO, s_l, m_run, s_flag, b, kvh, rg, split, nsplit, nrows, warp, lane,
+    tc_finish<RG, H::kRS, !FP8>(a, sO, s_l, m_run, s_flag, b, kvh, rg, split, nsplit, nrows, warp, lane,
                         tid, ok, (int64_t)b * gridDim.y + blockIdx.y);
 }
 
@@ -1512,7 +1530,7 @@ k_decode_i8(const TcArgs a)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
-    tc_finish<RG>(a, sO, s_l, m_run, s_flag, b, kvh, rg, split, nsplit, nrows, warp, lane, tid,
+    tc_finish<RG, 16>(a, sO, s_l, m_run, s_flag, b, kvh, rg, split, nsplit, nrows, warp, lane, tid,
                   ok, (int64_t)b * gridDim.y + blockIdx.y);
 }
 
@@ -1520,7 +1538,7 @@ template <int BITS, int RG, bool FP8 = false>
 cudaError_t launch_tc(const TcArgs& a, dim3 grid, cudaStream_t stream)
 {
     constexpr int NCOL = 2 * RG < 16 ? 16 : 2 * RG;
-    const size_t smem = 1536 + 2 * 256 * NCOL + (size_t)kStages * TcFmt<BITS, FP8>::kStage;
+    const size_t smem = TcHdr<RG>::kBytes + 2 * 256 * NCOL + (size_t)kStages * TcFmt<BITS, FP8>::kStage;
     static int configured = 0;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
