@@ -133,15 +133,25 @@ __device__ __forceinline__ void fwht32_across(float x[32], int q)
     }
 }
 
+// Smallest power of two >= 4 L, times 2^-24: the fast path's margin.
+__host__ __device__ constexpr float quant_margin(int L)
+{
+    float m = 1.f / 16777216.f;
+    for (int p = 1; p < 4 * L; p *= 2) m *= 2.f;
+    return m;
+}
+
 // Codes of this thread's 32 rotated values y (scale s): offset-binary
 // u = code + L with code = clamp(roundf(fl(y L) / s), -L, L), the division
-// an IEEE fp32 one.  Fast path: q = fl(fl(y L) * fl(1/s)) lies within 2^-15
-// of fl(fl(y L) / s) (|y L / s| <= L < 128, two roundings of relative size
-// 2^-24 each, plus the rounding of the quotient itself), so whenever q is
-// at least 2^-14 away from the nearest half-integer both round to the same
-// integer and rint(q) is the code.  Any value closer to a half-integer, a
-// non-finite q, or a scale outside [2^-125, 2^125] (where 1/s could lose
-// precision) sends the whole vector through the IEEE division.
+// an IEEE fp32 one.  Fast path: with t = fl(y L), |t / s| <= L (1 + 2^-24),
+// q = fl(t * fl(1/s)) and the IEEE quotient fl(t / s) each carry relative
+// rounding errors of at most 2^-24 (two for q, one for the quotient), so
+// they differ by less than 3.001 L 2^-24 < quant_margin(L).  Whenever q is
+// at least that margin away from the nearest half-integer both round to the
+// same integer (never beyond +-L), and rint(q) is the code.  Any value
+// closer to a half-integer, a non-finite q, or a scale outside
+// [2^-126, 2^125] (where 1/s could lose precision) sends the whole vector
+// through the IEEE division.
 template <int BITS>
 __device__ __forceinline__ void quantize32(const float y[32], float s, uint32_t u[32])
 {
@@ -161,6 +171,7 @@ __device__ __forceinline__ void quantize32(const float y[32], float s, uint32_t 
     constexpr uint32_t kBias = 0x4B400000u - (uint32_t)L; // bits(kRound + n) - kBias = n + L
     const unsigned long long L2 = pk2((float)L, (float)L), r2 = pk2(r, r);
     const unsigned long long m2 = pk2(kRound, kRound);
+    constexpr float kThr = 0.5f - quant_margin(L);          // exact in fp32
 #pragma unroll
     for (int i = 0; i < 32; i += 2) {
         const unsigned long long t2 = mul2(pk2(y[i], y[i + 1]), L2);
@@ -168,7 +179,7 @@ __device__ __forceinline__ void quantize32(const float y[32], float s, uint32_t 
         const unsigned long long n2 = add2(q2, m2);          // kRound + rint(q)
         float d0, d1, n0, n1;
         up2(sub2(q2, sub2(n2, m2)), d0, d1);                  // q - rint(q), exact
-        slow |= !(fabsf(d0) <= 0.49993896484375f) | !(fabsf(d1) <= 0.49993896484375f);  // 0.5 - 2^-14
+        slow |= !(fabsf(d0) <= kThr) | !(fabsf(d1) <= kThr);
         up2(n2, n0, n1);
         u[i] = __float_as_uint(n0) - kBias;
         u[i + 1] = __float_as_uint(n1) - kBias;
