@@ -40,10 +40,12 @@ constexpr int kQaThreads = 256;
 constexpr int kQaWin = 64;             // tokens per window before alignment (large calls)
 constexpr int kQaMaxWin = 128;         // staging capacity: kQaWin + page_size - 1 <= 127
 constexpr int kQaPass = 32;            // tokens per pass (x K and V = 64 vectors)
-// staging row: window tokens, XOR 8 (dim / 32), + one group (>= 160); 168 so
-// that the V writer's 8-byte reads of rows 2 apart spread over the banks
-constexpr int kVRow = 168;
-constexpr int kQaStages = 3;           // input ring: each thread's next passes, by cp.async
+// staging row: window tokens (< 128, XOR 8 (dim / 32) stays below 128) and
+// 8 bytes of pitch so that the V writer's 8-byte reads of rows 2 apart
+// spread over the banks; two buffers, so that the writer of one head runs
+// while the next head is quantised
+constexpr int kVRow = 136;
+constexpr int kQaStages = 2;           // input ring: each thread's next pass, by cp.async
 constexpr int kQaInBytes = kQaStages * kQaThreads * 64;
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem)
@@ -247,7 +249,7 @@ k_quantize_append(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v
 {
     constexpr int CB = kHeadDim * BITS / 8;            // K row bytes
     extern __shared__ __align__(16) uint8_t s_in[];    // [stage][chunk][thread][16 B] input ring
-    __shared__ __align__(16) uint8_t s_v[kHeadDim * kVRow];   // [dim][token ^ 8 (dim / 32)]
+    __shared__ __align__(16) uint8_t s_v[2][kHeadDim * kVRow];   // [head & 1][dim][token ^ 8 (dim / 32)]
     __shared__ int s_page[kQaMaxWin], s_off[kQaMaxWin], s_run[kQaMaxWin];
     __shared__ int s_rs[kQaMaxWin], s_rlen[kQaMaxWin];  // runs: first window token, length
     __shared__ int s_ritem[kQaMaxWin + 1];              // runs: first V work item
@@ -339,7 +341,7 @@ k_quantize_append(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v
         if (tid == kQaThreads - 1) s_ritem[kQaMaxWin] = before + x;     // total
         __syncthreads();
     }
-    auto write_v_rows = [&](int head) {
+    auto write_v_rows = [&](int head, const uint8_t* sv) {
     const int total = s_ritem[kQaMaxWin];
     for (int item = tid; item < total; item += kQaThreads) {
         int lo = 0, hi = nrun - 1;                       // the run: last s_ritem[r] <= item
@@ -360,7 +362,7 @@ k_quantize_append(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v
             const int f0 = kUnitFields * sub;
             auto group8 = [&](int f, uint32_t& lo4, uint32_t& hi4) {
                 const int d = f / P, off = f - d * P;
-                const uint8_t* row = s_v + d * kVRow;
+                const uint8_t* row = sv + d * kVRow;
                 const int x8 = 8 * (d >> 5), c = rs + off, a = c & ~7, o = c & 7;
                 const uint2 A = *reinterpret_cast<const uint2*>(row + (a ^ x8));
                 if (o == 0) {
@@ -447,7 +449,7 @@ k_quantize_append(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v
                     cw = w;
                     val = msk = 0;
                 }
-                const uint32_t uu = s_v[d * kVRow + ((rs + f) ^ (8 * (d >> 5)))];
+                const uint32_t uu = sv[d * kVRow + ((rs + f) ^ (8 * (d >> 5)))];
                 val |= uu << sh;
                 msk |= fm << sh;
                 if (sh + BITS > 32) {                 // a 3-bit field across two words
@@ -462,8 +464,8 @@ k_quantize_append(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v
     }
     };
     // ---- quantise: passes of 32 tokens of one head, warps 0-3 K, warps 4-7 V;
-    // each thread fetches its 64 input bytes of the next two passes by
-    // cp.async into its own slot of a 3-stage ring while it computes this one
+    // each thread fetches its 64 input bytes of the next pass by cp.async
+    // into its own slot of a 2-stage ring while it computes this one
     const int which = warp >> 2;
     const int q = lane & 3;
     const int vi = (warp & 3) * 8 + (lane >> 2);        // vector of the pass (token in chunk)
@@ -483,11 +485,11 @@ k_quantize_append(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v
         }
         cp_async_commit();
     };
-    issue(0);
-    issue(1);
+#pragma unroll
+    for (int p = 0; p < kQaStages - 1; ++p) issue(p);
     for (int pidx = 0; pidx < npass; ++pidx) {
-        issue(pidx + 2);
-        cp_async_wait<2>();                              // this pass's bytes have landed
+        issue(pidx + kQaStages - 1);
+        cp_async_wait<kQaStages - 1>();                  // this pass's bytes have landed
         const int hh = pidx / nchunk, chunk = pidx - hh * nchunk;
         const int head = head0 + hh;
         const int tk = chunk * kQaPass + vi;                                  // window token
@@ -577,13 +579,15 @@ k_quantize_append(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v
             } else {
                 // V: stage u dimension-major, column tk ^ 8q
 #pragma unroll
-                for (int i = 0; i < 32; ++i) s_v[(32 * q + i) * kVRow + (tk ^ (8 * q))] = (uint8_t)u[i];
+                for (int i = 0; i < 32; ++i)
+                    s_v[hh & 1][(32 * q + i) * kVRow + (tk ^ (8 * q))] = (uint8_t)u[i];
             }
         }
         if (chunk == nchunk - 1) {
-            __syncthreads();                             // head `head` is staged
-            write_v_rows(head);
-            __syncthreads();                             // the staging is free again
+            // head `head` is staged, and every thread is done writing the
+            // previous head from the other buffer, which the next head fills
+            __syncthreads();
+            write_v_rows(head, s_v[hh & 1]);
         }
     }
     cp_async_wait<0>();
